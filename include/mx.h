@@ -1,0 +1,173 @@
+/*
+ * libmx -- MXFP8 quantize, scale layout, block-scaled GEMM and grid equality on NVIDIA B200
+ * (sm_100a). C ABI: plain pointers and sizes; no allocation, no host synchronisation (except
+ * mx_device_error), every call asynchronous on `stream`.
+ *
+ * The operations follow "End-to-End MXFP8 Reinforcement Learning on Blackwell: What Matching
+ * Buys, When It Pays Off, and How It Fails" (W. Zhang, arXiv 2610.34915):
+ *   - Figure 1: the learner computes with MXFP8 GEMMs over BF16 master weights; at every weight
+ *     synchronization the weights are quantized with the learner's own quantizer, so the sampler
+ *     receives the learner's grid, and the sampler re-derives its kernel layouts in place;
+ *   - Table 6: per micro-batch the MXFP8 path spends time in "MXFP8 quantization", "scale
+ *     rearrangement" and "GEMM";
+ *   - Table 10 (F3, F4, F6) and Table 11 (byte comparison): the synchronized weight, scale and
+ *     kernel layout must equal the learner's quantization byte for byte.
+ * The pages do not print the quantization rule or the scale layout. The rule is the OCP MX v1.0
+ * one for MXFP8, the layout NVIDIA's sm_100 block-scaling-factor layout:
+ *   - elements: FP8 E4M3 ("fn": max 448, no infinities, S.1111.111 = NaN);
+ *   - one E8M0 scale per 32 consecutive elements along K: e = floor(log2(amax)) - 8, clamped to
+ *     [-127, 127], stored as e + 127; an all-zero block gets byte 0;
+ *   - element = round-to-nearest-even(x * 2^-e), saturated to +-448, signed zero kept;
+ *   - a block containing NaN or +-Inf gets scale 0xFF and every element byte sign | 0x7F;
+ *   - tensor-core scale layout: pad a [R, C] scale matrix to R' = ceil(R/128)*128 rows and
+ *     C' = ceil(C/4)*4 columns (pad bytes 0x00); 128 x 4 blocks of 512 bytes, row-block major;
+ *     inside a block, scale (r, c) is at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+ *
+ * Memory: the caller allocates and owns every buffer. All buffers named "device" must be device
+ * memory of the current CUDA device; all of them must be 16-byte aligned. Buffers must not
+ * overlap unless stated.
+ *
+ * Errors: arguments are checked on the host before any launch and reported as mx_status; nothing
+ * is launched when a check fails. MX_ERR_CUDA reports a failed launch or driver call. Device-side
+ * faults that a kernel detects (a bounded wait that expired, invalid grouped-GEMM row offsets)
+ * set bits in a device status word readable with mx_device_error.
+ */
+#ifndef MX_H
+#define MX_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* mx_stream;
+
+typedef enum {
+    MX_OK = 0,
+    MX_ERR_ARG = -1,          /* null pointer, negative size, bad flag or enum value */
+    MX_ERR_SHAPE = -2,        /* a size the operation cannot take (e.g. K % 32 != 0) */
+    MX_ERR_ALIGN = -3,        /* pointer or leading dimension not 16-byte aligned */
+    MX_ERR_CUDA = -4,         /* a CUDA launch or driver call failed */
+    MX_ERR_UNSUPPORTED = -5,  /* device is not sm_100 / feature unavailable */
+    MX_ERR_DEVICE = -6        /* mx_device_error found a device-side error bit set */
+} mx_status;
+
+/* mx_quantize flags. */
+enum { MX_ROWWISE = 1, MX_COLWISE = 2, MX_SWIZZLE = 4 };
+
+/* GEMM output element type. */
+typedef enum { MX_OUT_F32 = 0, MX_OUT_BF16 = 1 } mx_out_dtype;
+
+/* Bytes of the tensor-core scale layout for a [rows, kblocks] scale matrix:
+ * ceil(rows/128)*128 * ceil(kblocks/4)*4. Returns -1 for negative sizes. */
+int64_t mx_swizzled_scale_bytes(int64_t rows, int64_t kblocks);
+
+/*
+ * MXFP8 quantization of a BF16 matrix x[M, K] (device, row stride ld_x elements), the learner's
+ * quantizer of Figure 1 and Table 6 ("MXFP8 quantization"), with the scale rearrangement of
+ * Table 6 fused when MX_SWIZZLE is set. One pass over x produces any of:
+ *   MX_ROWWISE: q_row[M, K] E4M3 codes (packed, row stride K) and s_row, the E8M0 scales of the
+ *               32-blocks along K: raw [M, K/32] (packed), or with MX_SWIZZLE the tensor-core
+ *               layout of that matrix (mx_swizzled_scale_bytes(M, K/32) bytes, pads written 0).
+ *   MX_COLWISE: q_col[K, M] = the rowwise quantization of x^T (blocks of 32 along M, stored
+ *               K-major for the transposed GEMM operands of dgrad / wgrad) and s_col: raw
+ *               [K, M/32] or swizzled (mx_swizzled_scale_bytes(K, M/32) bytes).
+ * Requirements: K % 32 == 0; M % 32 == 0 if MX_COLWISE; ld_x >= K and ld_x % 8 == 0; at least
+ * one of MX_ROWWISE / MX_COLWISE; the pointers of each requested direction non-NULL (others are
+ * ignored); all pointers 16-byte aligned. M == 0 or K == 0 is a no-op.
+ * Result is bit-exact to the rule in the header comment.
+ */
+mx_status mx_quantize(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, int flags,
+                      uint8_t* q_row, uint8_t* s_row, uint8_t* q_col, uint8_t* s_col,
+                      mx_stream stream);
+
+/*
+ * Scale rearrangement (Table 6, "scale rearrangement"; Table 10 F3, the interleaved scale copy a
+ * backend derives): raw scales s[rows, kblocks] (device, packed) -> the tensor-core layout in
+ * s_swz (device). With group_rows_host == NULL the whole matrix is one group
+ * (mx_swizzled_scale_bytes(rows, kblocks) bytes). Otherwise group_rows_host (host memory, read
+ * during the call) lists `groups` consecutive row counts summing to `rows`; every group is padded
+ * to a multiple of 128 rows on its own and the groups' layouts are concatenated
+ * (sum_g ceil(rows_g/128)*128 * ceil(kblocks/4)*4 bytes) -- the A-operand scale layout that
+ * mx_grouped_gemm reads. Pad bytes are written 0.
+ */
+mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks,
+                            const int64_t* group_rows_host, int64_t groups, uint8_t* s_swz,
+                            mx_stream stream);
+
+/*
+ * Dense block-scaled MXFP8 GEMM (Table 6, "GEMM"): C[M, N] = A . B^T with
+ * A[m, k] = dec(qa[m, k]) * 2^(sa[m, k/32] - 127) and B[n, k] likewise, accumulated in fp32 on
+ * the tensor cores and written as fp32 or BF16 (round-to-nearest-even).
+ *   qa[M, K], qb[N, K]: E4M3 codes, K-major, packed (device);
+ *   sa_swz, sb_swz: scales of qa and qb in the tensor-core layout (as mx_quantize with
+ *                   MX_SWIZZLE writes them) (device);
+ *   c: device, row stride ld_c elements; rows >= M / columns >= N are never written.
+ * Requirements: M, N >= 0, K > 0, K % 32 == 0, ld_c >= N, ld_c * sizeof(out) % 16 == 0, all
+ * pointers 16-byte aligned, M, N, K < 2^31.
+ * Accuracy: |c - exact| <= 1e-5 * sum_k |a_k b_k| (+ 2^-8 |exact| for BF16 output).
+ */
+mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz,
+                  int64_t M, int64_t N, int64_t K, void* c, int64_t ld_c, mx_out_dtype out_dtype,
+                  mx_stream stream);
+
+/*
+ * Grouped block-scaled MXFP8 GEMM for MoE experts (Table 2: Qwen3-30B-A3B, 128 experts, top-8;
+ * Table 10 F4, the sampler's expert layout). For every group g, rows [off[g], off[g+1]) of A
+ * are multiplied with expert weight B_g:  C[r, :] = A[r, :] . B_g^T.
+ *   qa[total_rows, K]: E4M3 codes, rows grouped by expert (device);
+ *   sa_swz: A's scales in the grouped tensor-core layout (mx_swizzle_scales with the groups'
+ *           row counts: each group padded to 128 rows) (device);
+ *   qb[G, N, K]: expert weights (device); sb_swz: G consecutive tensor-core layouts of the
+ *           experts' [N, K/32] scales, mx_swizzled_scale_bytes(N, K/32) bytes each (device);
+ *   row_offsets_dev[G + 1]: int32 device array, 0 = off[0] <= off[1] <= ... <= off[G] =
+ *           total_rows. The host never reads it; invalid offsets set a device error bit and no
+ *           output is written;
+ *   c: device, [total_rows, N] with row stride ld_c.
+ * Requirements: 1 <= G <= 1024 and those of mx_gemm.
+ */
+mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
+                          const uint8_t* sb_swz, const int32_t* row_offsets_dev, int64_t G,
+                          int64_t total_rows, int64_t N, int64_t K, void* c, int64_t ld_c,
+                          mx_out_dtype out_dtype, mx_stream stream);
+
+/*
+ * Byte comparison (abstract and Table 11: the synchronized sampler weights, scales and kernel
+ * layout must equal the learner's quantization byte for byte): counts the positions i < nbytes
+ * with a[i] != b[i] and finds the smallest such i. Results are written to device memory:
+ * *mismatches_dev (uint64) and *first_index_dev (int64, -1 if none); both are overwritten.
+ * a, b: device buffers (any alignment; 16-byte aligned ones take the vector path).
+ */
+mx_status mx_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes,
+                        unsigned long long* mismatches_dev, long long* first_index_dev,
+                        mx_stream stream);
+
+/* Human-readable name of a status code (static string). */
+const char* mx_status_string(mx_status status);
+
+/*
+ * Reads and clears the device status word of the current device (synchronizes the device).
+ * *bits receives the error bits (1: a bounded wait expired; 2: invalid grouped-GEMM row offsets).
+ * Returns MX_OK when no bit was set, MX_ERR_DEVICE when some bit was set, MX_ERR_CUDA on failure.
+ */
+mx_status mx_device_error(uint32_t* bits);
+
+/*
+ * Deadline of every bounded wait inside libmx kernels, in nanoseconds (default 2e9 = 2 s); 0
+ * restores the default. Affects launches made after the call.
+ */
+void mx_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Diagnostic: launches one block whose thread waits on an mbarrier that nothing ever completes,
+ * under the current wait deadline. The wait expires, the kernel records error bit 1 and
+ * returns; read it with mx_device_error. Used to test that expired waits end a kernel cleanly.
+ */
+mx_status mx_diag_expired_wait(mx_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MX_H */

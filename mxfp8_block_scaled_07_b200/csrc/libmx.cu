@@ -1,0 +1,379 @@
+// libmx: the C-ABI entry points declared in include/mx.h. Host-side argument checks, tensor-map
+// construction and kernel launches; the kernels themselves are in quantize.cuh, grid_equal.cuh
+// and gemm.cuh. Nothing here allocates device memory or synchronizes (except mx_device_error).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mx.h"
+#include "gemm.cuh"
+#include "grid_equal.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace mx {
+
+// Device status word: error bits set by kernels (expired bounded waits, bad grouped offsets).
+__device__ uint32_t g_status_word;
+
+__global__ void expired_wait_kernel(uint32_t* err, uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // Nothing arrives on `bar`: the wait must expire, record the error and return.
+    mbar_wait(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), err, timeout_ns);
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+struct DeviceInfo {
+    int sms = 0;
+    int cc_major = 0;
+    uint32_t* status = nullptr;
+    int quant_blocks_per_sm[4] = {0, 0, 0, 0};
+    bool gemm_attr_set = false;
+    bool ok = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+template <bool R, bool C>
+int quant_occupancy() {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<R, C>, kQThreads, 0);
+    return n > 0 ? n : 1;
+}
+
+// Per-device facts, queried once with that device current.
+const DeviceInfo* device_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ok) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+        if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return nullptr;
+        if (d.cc_major != 10) {
+            d.ok = true;   // remembered as unsupported
+            return &d;
+        }
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        d.status = static_cast<uint32_t*>(p);
+        d.quant_blocks_per_sm[1] = quant_occupancy<true, false>();
+        d.quant_blocks_per_sm[2] = quant_occupancy<false, true>();
+        d.quant_blocks_per_sm[3] = quant_occupancy<true, true>();
+        if (cudaFuncSetAttribute(mx_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemDense) != cudaSuccess ||
+            cudaFuncSetAttribute(mx_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemGrouped) != cudaSuccess)
+            return nullptr;
+        d.ok = true;
+    }
+    return &d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mx_status check_device(const DeviceInfo** out) {
+    const DeviceInfo* d = device_info();
+    if (!d) return MX_ERR_CUDA;
+    if (d->cc_major != 10) return MX_ERR_UNSUPPORTED;
+    *out = d;
+    return MX_OK;
+}
+
+mx_status launched() { return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
+
+bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t rows, uint32_t box_cols,
+               uint32_t box_rows) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode) return false;
+    const cuuint64_t dims[2] = {cols_bytes, rows};
+    const cuuint64_t strides[1] = {cols_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Checks shared by both GEMMs. Sets *empty when there is nothing to compute (then pointers may be
+// null). The output may have any element alignment; 16-byte aligned rows take vector stores.
+mx_status gemm_checks(const void* qa, const void* sa, const void* qb, const void* sb, int64_t M, int64_t N,
+                      int64_t K, const void* c, int64_t ld_c, mx_out_dtype dt, bool* empty) {
+    if (M < 0 || N < 0 || K <= 0 || (dt != MX_OUT_F32 && dt != MX_OUT_BF16)) return MX_ERR_ARG;
+    if (K % 32 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MX_ERR_SHAPE;
+    if (ld_c < N) return MX_ERR_SHAPE;
+    *empty = (M == 0 || N == 0);
+    if (*empty) return MX_OK;
+    if (!qa || !sa || !qb || !sb || !c) return MX_ERR_ARG;
+    const int64_t esz = dt == MX_OUT_BF16 ? 2 : 4;
+    if (!aligned16(qa) || !aligned16(sa) || !aligned16(qb) || !aligned16(sb) ||
+        (reinterpret_cast<uintptr_t>(c) % esz) != 0)
+        return MX_ERR_ALIGN;
+    return MX_OK;
+}
+
+int vector_store_ok(const void* c, int64_t ld_c, mx_out_dtype dt) {
+    const int64_t esz = dt == MX_OUT_BF16 ? 2 : 4;
+    return aligned16(c) && (ld_c * esz) % 16 == 0;
+}
+
+}  // namespace
+}  // namespace mx
+
+using namespace mx;
+
+extern "C" {
+
+int64_t mx_swizzled_scale_bytes(int64_t rows, int64_t kblocks) {
+    if (rows < 0 || kblocks < 0) return -1;
+    return ceil_div(rows, 128) * 128 * (ceil_div(kblocks, 4) * 4);
+}
+
+const char* mx_status_string(mx_status s) {
+    switch (s) {
+        case MX_OK: return "MX_OK";
+        case MX_ERR_ARG: return "MX_ERR_ARG: invalid argument";
+        case MX_ERR_SHAPE: return "MX_ERR_SHAPE: unsupported shape";
+        case MX_ERR_ALIGN: return "MX_ERR_ALIGN: pointer or stride not 16-byte aligned";
+        case MX_ERR_CUDA: return "MX_ERR_CUDA: CUDA launch or driver call failed";
+        case MX_ERR_UNSUPPORTED: return "MX_ERR_UNSUPPORTED: device is not sm_100";
+        case MX_ERR_DEVICE: return "MX_ERR_DEVICE: a kernel reported a device-side error";
+    }
+    return "unknown mx_status";
+}
+
+void mx_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs); }
+
+mx_status mx_device_error(uint32_t* bits) {
+    if (!bits) return MX_ERR_ARG;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    uint32_t v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MX_ERR_CUDA;
+    if (cudaMemcpy(&v, d->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MX_ERR_CUDA;
+    const uint32_t zero = 0;
+    if (cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return MX_ERR_CUDA;
+    *bits = v;
+    return v ? MX_ERR_DEVICE : MX_OK;
+}
+
+mx_status mx_diag_expired_wait(mx_stream stream) {
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    expired_wait_kernel<<<1, 32, 0, stream>>>(d->status, g_timeout_ns.load());
+    return launched();
+}
+
+mx_status mx_quantize(const void* x, int64_t M, int64_t K, int64_t ld_x, int flags, uint8_t* q_row,
+                      uint8_t* s_row, uint8_t* q_col, uint8_t* s_col, mx_stream stream) {
+    const bool row = flags & MX_ROWWISE, col = flags & MX_COLWISE, swz = flags & MX_SWIZZLE;
+    if (flags & ~(MX_ROWWISE | MX_COLWISE | MX_SWIZZLE)) return MX_ERR_ARG;
+    if (!row && !col) return MX_ERR_ARG;
+    if (M < 0 || K < 0) return MX_ERR_ARG;
+    if (K % 32 != 0 || (col && M % 32 != 0)) return MX_ERR_SHAPE;
+    if (M == 0 || K == 0) return MX_OK;   // empty tensors may carry null pointers
+    if (!x || (row && (!q_row || !s_row)) || (col && (!q_col || !s_col))) return MX_ERR_ARG;
+    if (ld_x < K) return MX_ERR_SHAPE;
+    if (!aligned16(x) || ld_x % 8 != 0) return MX_ERR_ALIGN;
+    if (row && (!aligned16(q_row) || !aligned16(s_row))) return MX_ERR_ALIGN;
+    if (col && (!aligned16(q_col) || !aligned16(s_col))) return MX_ERR_ALIGN;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+
+    QuantArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.M = M;
+    a.K = K;
+    a.ldx = ld_x;
+    a.q_row = q_row;
+    a.s_row = s_row;
+    a.q_col = q_col;
+    a.s_col = s_col;
+    a.swz_row = swz;
+    a.swz_col = swz;
+    a.tiles_m = ceil_div(M, kQTile);
+    a.tiles_k = ceil_div(K, kQTile);
+    a.tiles = a.tiles_m * a.tiles_k;
+    const int which = (row ? 1 : 0) | (col ? 2 : 0);
+    const int64_t grid = std::min<int64_t>(a.tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
+    if (row && col)
+        quantize_kernel<true, true><<<grid, kQThreads, 0, stream>>>(a);
+    else if (row)
+        quantize_kernel<true, false><<<grid, kQThreads, 0, stream>>>(a);
+    else
+        quantize_kernel<false, true><<<grid, kQThreads, 0, stream>>>(a);
+    return launched();
+}
+
+mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, const int64_t* group_rows_host,
+                            int64_t groups, uint8_t* s_swz, mx_stream stream) {
+    if (!s || !s_swz || rows < 0 || kblocks < 0) return MX_ERR_ARG;
+    if (group_rows_host && groups < 1) return MX_ERR_ARG;
+    if (!aligned16(s_swz)) return MX_ERR_ALIGN;
+    if (group_rows_host) {
+        int64_t total = 0;
+        for (int64_t g = 0; g < groups; ++g) {
+            if (group_rows_host[g] < 0) return MX_ERR_ARG;
+            total += group_rows_host[g];
+        }
+        if (total != rows) return MX_ERR_SHAPE;
+    }
+    if (rows == 0 || kblocks == 0) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+
+    const int64_t one = rows;
+    const int64_t* gr = group_rows_host ? group_rows_host : &one;
+    const int64_t ng = group_rows_host ? groups : 1;
+    const int64_t ctiles = ceil_div(kblocks, 4);
+    int64_t src_row = 0, out_block = 0;
+    for (int64_t g0 = 0; g0 < ng; g0 += kSwzMaxGroups) {
+        SwizzleArgs a;
+        a.s = s;
+        a.kblocks = kblocks;
+        a.ctiles = ctiles;
+        a.ngroups = static_cast<int>(std::min<int64_t>(kSwzMaxGroups, ng - g0));
+        a.out = s_swz + out_block * 512;
+        int64_t local_block = 0;
+        for (int i = 0; i < a.ngroups; ++i) {
+            a.src_row[i] = src_row;
+            a.rows[i] = gr[g0 + i];
+            a.block_start[i] = local_block;
+            local_block += ceil_div(gr[g0 + i], 128) * ctiles;
+            src_row += gr[g0 + i];
+        }
+        a.block_start[a.ngroups] = local_block;
+        if (local_block > 0) {
+            const int64_t warps = local_block;
+            const int64_t grid = std::min<int64_t>(ceil_div(warps * 32, 256), int64_t(d->sms) * 16);
+            swizzle_kernel<<<grid, 256, 0, stream>>>(a);
+            if (mx_status st = launched()) return st;
+        }
+        out_block += local_block;
+    }
+    return MX_OK;
+}
+
+mx_status mx_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes, unsigned long long* mismatches_dev,
+                        long long* first_index_dev, mx_stream stream) {
+    if (!mismatches_dev || !first_index_dev || nbytes < 0 || (nbytes > 0 && (!a || !b))) return MX_ERR_ARG;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    grid_equal_reset_kernel<<<1, 1, 0, stream>>>(mismatches_dev, first_index_dev);
+    if (mx_status st = launched()) return st;
+    if (nbytes == 0) return MX_OK;
+    const int vec = aligned16(a) && aligned16(b);
+    const int64_t work = vec ? ceil_div(nbytes, 16 * kGeUnroll) : nbytes;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(work, kGeThreads), int64_t(d->sms) * 8));
+    grid_equal_kernel<<<grid, kGeThreads, 0, stream>>>(a, b, nbytes, vec, mismatches_dev, first_index_dev);
+    return launched();
+}
+
+mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz, int64_t M,
+                  int64_t N, int64_t K, void* c, int64_t ld_c, mx_out_dtype out_dtype, mx_stream stream) {
+    bool empty = false;
+    if (mx_status st = gemm_checks(qa, sa_swz, qb, sb_swz, M, N, K, c, ld_c, out_dtype, &empty)) return st;
+    if (empty) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, qa, K, M, kBK, kBM) || !make_tmap(&tb, qb, K, N, kBK, kBN)) return MX_ERR_CUDA;
+    GemmArgs a{};
+    a.sfa = sa_swz;
+    a.sfb = sb_swz;
+    a.c = c;
+    a.ldc = ld_c;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.nkb = static_cast<int>(ceil_div(K, kBK));
+    a.tiles_m = static_cast<int>(ceil_div(M, kBM));
+    a.tiles_n = static_cast<int>(ceil_div(N, kBN));
+    a.out_bf16 = out_dtype == MX_OUT_BF16;
+    a.vec_store = vector_store_ok(c, ld_c, out_dtype);
+    a.G = 1;
+    a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
+    a.row_offsets = nullptr;
+    a.err = d->status;
+    a.timeout_ns = g_timeout_ns.load();
+    const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, d->sms));
+    mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, a);
+    return launched();
+}
+
+mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz,
+                          const int32_t* row_offsets_dev, int64_t G, int64_t total_rows, int64_t N, int64_t K,
+                          void* c, int64_t ld_c, mx_out_dtype out_dtype, mx_stream stream) {
+    if (!row_offsets_dev || G < 1) return MX_ERR_ARG;
+    if (G > kMaxGroups) return MX_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(row_offsets_dev) & 3u) return MX_ERR_ALIGN;
+    bool empty = false;
+    if (mx_status st = gemm_checks(qa, sa_swz, qb, sb_swz, total_rows, N, K, c, ld_c, out_dtype, &empty))
+        return st;
+    if (G * N >= (int64_t(1) << 31)) return MX_ERR_SHAPE;
+    if (empty) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN))
+        return MX_ERR_CUDA;
+    GemmArgs a{};
+    a.sfa = sa_swz;
+    a.sfb = sb_swz;
+    a.c = c;
+    a.ldc = ld_c;
+    a.M = static_cast<int>(total_rows);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.nkb = static_cast<int>(ceil_div(K, kBK));
+    a.tiles_m = 0;
+    a.tiles_n = static_cast<int>(ceil_div(N, kBN));
+    a.out_bf16 = out_dtype == MX_OUT_BF16;
+    a.vec_store = vector_store_ok(c, ld_c, out_dtype);
+    a.G = static_cast<int>(G);
+    a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
+    a.row_offsets = row_offsets_dev;
+    a.err = d->status;
+    a.timeout_ns = g_timeout_ns.load();
+    // Upper bound on tiles: every group adds at most one partial 128-row tile.
+    const int64_t max_tiles = (ceil_div(total_rows, kBM) + G) * a.tiles_n;
+    const int grid = static_cast<int>(std::min<int64_t>(max_tiles, d->sms));
+    mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, a);
+    return launched();
+}
+
+}  // extern "C"

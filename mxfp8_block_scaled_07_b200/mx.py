@@ -1,0 +1,180 @@
+"""Thin Python binding of libmx (include/mx.h) over ctypes.
+
+Argument marshalling only: every step runs in the CUDA kernels of ``libmx.so``. PyTorch
+supplies device memory (output tensors are allocated with ``torch.empty`` on the input's
+device) and the current stream. There is no fallback: if ``libmx.so`` is missing or a call
+fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmx.so")
+
+MX_ROWWISE, MX_COLWISE, MX_SWIZZLE = 1, 2, 4
+MX_OUT_F32, MX_OUT_BF16 = 0, 1
+_STATUS = {0: "MX_OK", -1: "MX_ERR_ARG", -2: "MX_ERR_SHAPE", -3: "MX_ERR_ALIGN", -4: "MX_ERR_CUDA",
+           -5: "MX_ERR_UNSUPPORTED", -6: "MX_ERR_DEVICE"}
+
+_lib = None
+
+
+class MxError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmx.so with argument types declared (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmx.so not built ({LIB_PATH}); run python -m mxfp8_block_scaled_07_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64
+    L.mx_swizzled_scale_bytes.argtypes = [I64, I64]
+    L.mx_swizzled_scale_bytes.restype = I64
+    L.mx_quantize.argtypes = [P, I64, I64, I64, I32, P, P, P, P, P]
+    L.mx_quantize.restype = I32
+    L.mx_swizzle_scales.argtypes = [P, I64, I64, P, I64, P, P]
+    L.mx_swizzle_scales.restype = I32
+    L.mx_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, I32, P]
+    L.mx_gemm.restype = I32
+    L.mx_grouped_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, I32, P]
+    L.mx_grouped_gemm.restype = I32
+    L.mx_grid_equal.argtypes = [P, P, I64, P, P, P]
+    L.mx_grid_equal.restype = I32
+    L.mx_status_string.argtypes = [I32]
+    L.mx_status_string.restype = ctypes.c_char_p
+    L.mx_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    L.mx_device_error.restype = I32
+    L.mx_set_wait_timeout_ns.argtypes = [U64]
+    L.mx_set_wait_timeout_ns.restype = None
+    L.mx_diag_expired_wait.argtypes = [P]
+    L.mx_diag_expired_wait.restype = I32
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MxError(status, what)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def swizzled_scale_bytes(rows: int, kblocks: int) -> int:
+    return int(lib().mx_swizzled_scale_bytes(rows, kblocks))
+
+
+def grouped_swizzled_scale_bytes(group_rows, kblocks: int) -> int:
+    return sum(swizzled_scale_bytes(int(r), kblocks) for r in group_rows)
+
+
+def quantize(x: torch.Tensor, rowwise: bool = True, colwise: bool = False, swizzle: bool = True, out=None):
+    """mx_quantize on a 2-D BF16 CUDA tensor. Returns (q_row, s_row, q_col, s_col); entries of a
+    direction not requested are None. ``out`` may supply the four buffers."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    flags = (MX_ROWWISE if rowwise else 0) | (MX_COLWISE if colwise else 0) | (MX_SWIZZLE if swizzle else 0)
+    dev = x.device
+    if out is None:
+        u8 = dict(dtype=torch.uint8, device=dev)
+        q_row = torch.empty((M, K), **u8) if rowwise else None
+        s_row = (torch.empty(swizzled_scale_bytes(M, K // 32), **u8) if swizzle
+                 else torch.empty((M, K // 32), **u8)) if rowwise else None
+        q_col = torch.empty((K, M), **u8) if colwise else None
+        s_col = (torch.empty(swizzled_scale_bytes(K, M // 32), **u8) if swizzle
+                 else torch.empty((K, M // 32), **u8)) if colwise else None
+    else:
+        q_row, s_row, q_col, s_col = out
+    st = lib().mx_quantize(_p(x), M, K, x.stride(0), flags, _p(q_row), _p(s_row), _p(q_col), _p(s_col),
+                           ctypes.c_void_p(_stream(dev)))
+    _check(st, "mx_quantize")
+    return q_row, s_row, q_col, s_col
+
+
+def swizzle_scales(s: torch.Tensor, group_rows=None, out=None):
+    """mx_swizzle_scales on raw scales [rows, kblocks] (uint8, CUDA)."""
+    assert s.dtype == torch.uint8 and s.dim() == 2 and s.is_contiguous()
+    rows, kb = s.shape
+    if group_rows is not None:
+        gr = [int(r) for r in group_rows]
+        size = grouped_swizzled_scale_bytes(gr, kb)
+        arr = (ctypes.c_int64 * len(gr))(*gr)
+        gptr, ng = ctypes.cast(arr, ctypes.c_void_p), len(gr)
+    else:
+        size, gptr, ng = swizzled_scale_bytes(rows, kb), None, 0
+    if out is None:
+        out = torch.empty(size, dtype=torch.uint8, device=s.device)
+    st = lib().mx_swizzle_scales(_p(s), rows, kb, gptr, ng, _p(out), ctypes.c_void_p(_stream(s.device)))
+    _check(st, "mx_swizzle_scales")
+    return out
+
+
+def _out_code(dtype) -> int:
+    return {torch.float32: MX_OUT_F32, torch.bfloat16: MX_OUT_BF16}[dtype]
+
+
+def gemm(qa, sa_swz, qb, sb_swz, out_dtype=torch.bfloat16, out=None):
+    """mx_gemm: C[M, N] = A . B^T from K-major E4M3 operands and tensor-core-layout scales."""
+    M, K = qa.shape
+    N = qb.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    st = lib().mx_gemm(_p(qa), _p(sa_swz), _p(qb), _p(sb_swz), M, N, K, _p(out), out.stride(0),
+                       _out_code(out.dtype), ctypes.c_void_p(_stream(qa.device)))
+    _check(st, "mx_gemm")
+    return out
+
+
+def grouped_gemm(qa, sa_swz, qb, sb_swz, row_offsets, out_dtype=torch.bfloat16, out=None):
+    """mx_grouped_gemm: rows [off[g], off[g+1]) of A against qb[g]. row_offsets: int32 CUDA [G+1]."""
+    total, K = qa.shape
+    G, N, K2 = qb.shape
+    assert K2 == K and row_offsets.dtype == torch.int32 and row_offsets.numel() == G + 1
+    if out is None:
+        out = torch.empty((total, N), dtype=out_dtype, device=qa.device)
+    st = lib().mx_grouped_gemm(_p(qa), _p(sa_swz), _p(qb), _p(sb_swz), _p(row_offsets), G, total, N, K, _p(out),
+                               out.stride(0), _out_code(out.dtype), ctypes.c_void_p(_stream(qa.device)))
+    _check(st, "mx_grouped_gemm")
+    return out
+
+
+def grid_equal(a: torch.Tensor, b: torch.Tensor, out=None):
+    """mx_grid_equal over the bytes of two CUDA tensors. Returns (mismatches, first_index) as
+    1-element int64 device tensors (no host synchronisation)."""
+    assert a.is_contiguous() and b.is_contiguous()
+    n = a.numel() * a.element_size()
+    assert b.numel() * b.element_size() == n
+    if out is None:
+        out = torch.empty(2, dtype=torch.int64, device=a.device)
+    cnt, first = out[0:1], out[1:2]
+    st = lib().mx_grid_equal(_p(a), _p(b), n, _p(cnt), _p(first), ctypes.c_void_p(_stream(a.device)))
+    _check(st, "mx_grid_equal")
+    return cnt, first
+
+
+def device_error() -> int:
+    """Reads and clears the device status word (synchronizes). 0 means no error bit set."""
+    bits = ctypes.c_uint32(0)
+    st = lib().mx_device_error(ctypes.byref(bits))
+    if st not in (0, -6):
+        _check(st, "mx_device_error")
+    return int(bits.value)
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().mx_set_wait_timeout_ns(int(ns))

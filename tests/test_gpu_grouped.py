@@ -1,0 +1,101 @@
+"""GPU parity: mx_swizzle_scales (single and grouped) bit-exact, and mx_grouped_gemm against the
+fp64 oracle within the GEMM tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_gemm_close, to_np
+from mxfp8_block_scaled_07_b200 import mx, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("rows,kb", [(1, 1), (128, 4), (300, 13), (1024, 64), (4097, 130)])
+def test_swizzle_single_group(rows, kb):
+    s = synth.random_bytes(rows * kb, seed=rows + kb).reshape(rows, kb)
+    out = mx.swizzle_scales(s.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(out), oracle.swizzle(s.numpy()))
+
+
+@pytest.mark.parametrize("groups", [[0, 5, 128, 129, 300, 0, 1], [7] * 200, [0], [256, 0, 0, 3]])
+def test_swizzle_grouped(groups):
+    kb = 64
+    rows = sum(groups)
+    s = synth.random_bytes(max(rows, 1) * kb, seed=len(groups))[: rows * kb].reshape(rows, kb)
+    if rows == 0:
+        pytest.skip("no rows")
+    out = mx.swizzle_scales(s.cuda(), groups)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(out), oracle.swizzle(s.numpy(), groups))
+
+
+def grouped_case(counts, N, K, out_dtype, seed=0, device_inputs=None):
+    counts = [int(c) for c in counts]
+    off = synth.group_offsets(counts)
+    G = len(counts)
+    rows = off[-1]
+    if device_inputs is None:
+        X = synth.normal_bf16((rows, K), seed=seed, outlier_frac=0.01, outlier_scale=100.0)
+        W = synth.normal_bf16((G, N, K), std=0.02, seed=seed + 1)
+    else:
+        X, W = device_inputs
+    Xd, Wd = X.cuda(), W.cuda()
+    qx, sx_raw, _, _ = mx.quantize(Xd, True, False, swizzle=False)
+    sx = mx.swizzle_scales(sx_raw, counts)
+    qw, sw, _, _ = mx.quantize(Wd.reshape(G * N, K), True, False, swizzle=True)
+    offs = torch.tensor(off, dtype=torch.int32, device="cuda")
+    c = mx.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw, offs, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return X, W, off, c
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_grouped_small_ragged_with_empty_groups(out_dtype):
+    counts = [0, 5, 128, 129, 300, 0, 1, 64]
+    N, K = 384, 256
+    X, W, off, c = grouped_case(counts, N, K, out_dtype, seed=3)
+    qx, sx = oracle.quantize_rowwise(X)
+    qw, sw = oracle.quantize_rowwise(W.reshape(-1, K))
+    ref, abs_sum = oracle.grouped_gemm(qx, sx, qw.reshape(len(counts), N, K), sw.reshape(len(counts), N, K // 32), off)
+    assert_gemm_close(to_np(c.float()), ref, abs_sum, out_dtype == torch.bfloat16, "grouped small")
+
+
+def test_grouped_bad_offsets_set_device_error_and_write_nothing():
+    counts = [64, 64]
+    N, K = 256, 128
+    X = synth.normal_bf16((128, K), seed=1).cuda()
+    W = synth.normal_bf16((2, N, K), seed=2).cuda()
+    qx, sx_raw, _, _ = mx.quantize(X, True, False, swizzle=False)
+    sx = mx.swizzle_scales(sx_raw, counts)
+    qw, sw, _, _ = mx.quantize(W.reshape(2 * N, K), True, False, swizzle=True)
+    mx.device_error()
+    bad = torch.tensor([0, 100, 64], dtype=torch.int32, device="cuda")      # decreasing, wrong total
+    out = torch.full((128, N), 3.0, device="cuda")
+    mx.grouped_gemm(qx, sx, qw.reshape(2, N, K), sw, bad, out=out)
+    assert mx.device_error() == 2
+    assert torch.all(out == 3.0)
+
+
+def test_moe_layer_full_size_sampled():
+    """Qwen3-30B-A3B MoE layer at full size: 163 840 routed rows (Zipf(1.1) top-8 over 128 experts),
+    gate_up (N 1536, K 2048) and down (N 2048, K 768), BF16 out; sampled rows of every expert."""
+    counts, Xp, H, W1, W2 = synth.moe_inputs(device="cuda")
+    counts = [int(c) for c in counts]
+    off = synth.group_offsets(counts)
+    G = len(counts)
+    g = np.random.default_rng(4)
+    for name, X, W in (("gate_up", Xp, W1), ("down", H, W2)):
+        N, K = W.shape[1], W.shape[2]
+        _, _, _, c = grouped_case(counts, N, K, torch.bfloat16, device_inputs=(X, W))
+        for e in range(G):
+            if counts[e] == 0:
+                continue
+            rr = np.unique(np.concatenate([[off[e], off[e + 1] - 1], off[e] + g.integers(0, counts[e], 2)]))
+            qa, sa = oracle.quantize_rowwise(X[torch.from_numpy(rr).cuda()].cpu())
+            cols = np.unique(g.integers(0, N, 96))
+            qb, sb = oracle.quantize_rowwise(W[e][torch.from_numpy(cols).cuda()].cpu())
+            ref, abs_sum = oracle.gemm(qa, sa, qb, sb)
+            assert_gemm_close(to_np(c[torch.from_numpy(rr).cuda()][:, torch.from_numpy(cols).cuda()].float()),
+                              ref, abs_sum, True, f"{name} expert {e}")
