@@ -216,41 +216,44 @@ class SyncWorkload:
             self.total_elems += W.numel()
             self.compare_bytes += 2 * (q.numel() + s.numel())
         torch.cuda.synchronize()
-        self.results = torch.zeros((len(self.items), 2, 2), dtype=torch.int64, device=device)
-        # Pre-marshalled C-ABI calls (plain pointers and sizes).
-        self.quant_calls = []
-        self.cmp_calls = []
-        P = ctypes.c_void_p
-        for i, (W, q, s, qs, ss) in enumerate(self.items):
-            M, K = W.shape
-            self.quant_calls.append((P(W.data_ptr()), M, K, K, 1 | 4, P(q.data_ptr()), P(s.data_ptr()), None, None))
-            r = self.results[i]
-            self.cmp_calls.append((P(q.data_ptr()), P(qs.data_ptr()), q.numel(), P(r[0, 0].data_ptr()),
-                                   P(r[0, 1].data_ptr())))
-            self.cmp_calls.append((P(s.data_ptr()), P(ss.data_ptr()), s.numel(), P(r[1, 0].data_ptr()),
-                                   P(r[1, 1].data_ptr())))
+        # Pair 2i: elements of tensor i; pair 2i + 1: its swizzled scales. results[0] = mismatch
+        # counts, results[1] = first indices.
+        self.results = torch.zeros((2, 2 * len(self.items)), dtype=torch.int64, device=device)
+        # Pre-marshalled C-ABI arguments (plain pointers and sizes): one multi-tensor quantization
+        # of all weights and one multi-pair byte comparison per step.
+        self.qarr = mx.quant_tensor_array([it[0] for it in self.items],
+                                          [(q, s, None, None) for (_, q, s, _, _) in self.items])
+        pairs = []
+        for (_, q, s, qs, ss) in self.items:
+            pairs += [(q, qs), (s, ss)]
+        self.parr = mx.compare_pair_array(pairs)
+        self.n_pairs = len(pairs)
         self.L = L
         self.quant_bytes = self.total_elems * QUANT_BYTES_PER_ELEM
         self.step_bytes = self.quant_bytes + self.compare_bytes
 
-    def launches_per_step(self):
-        return len(self.quant_calls) + 2 * len(self.cmp_calls)     # grid_equal = reset + compare
+    LAUNCHES_PER_STEP = 3      # mx_quantize_multi: 1 launch; mx_grid_equal_multi: reset + compare
+
+    def quantize_all(self, sp):
+        st = self.L.mx_quantize_multi(ctypes.cast(self.qarr, ctypes.c_void_p), len(self.items), 1 | 4, sp)
+        if st:
+            raise RuntimeError(f"mx_quantize_multi failed: {st}")
+
+    def compare_all(self, sp):
+        st = self.L.mx_grid_equal_multi(ctypes.cast(self.parr, ctypes.c_void_p), self.n_pairs,
+                                        ctypes.c_void_p(self.results[0].data_ptr()),
+                                        ctypes.c_void_p(self.results[1].data_ptr()), sp)
+        if st:
+            raise RuntimeError(f"mx_grid_equal_multi failed: {st}")
 
     def step(self, stream_ptr, ev_q0=None, ev_q1=None, ev_c1=None, stream=None):
-        L = self.L
         sp = ctypes.c_void_p(stream_ptr)
         if ev_q0 is not None:
             ev_q0.record(stream)
-        for args in self.quant_calls:
-            st = L.mx_quantize(*args, sp)
-            if st:
-                raise RuntimeError(f"mx_quantize failed: {st}")
+        self.quantize_all(sp)
         if ev_q1 is not None:
             ev_q1.record(stream)
-        for args in self.cmp_calls:
-            st = L.mx_grid_equal(*args, sp)
-            if st:
-                raise RuntimeError(f"mx_grid_equal failed: {st}")
+        self.compare_all(sp)
         if ev_c1 is not None:
             ev_c1.record(stream)
 
@@ -343,11 +346,9 @@ def run_e2e(wl, args, device):
     def one_step():
         for i, (W, q, s, qs, ss) in enumerate(wl.items):
             W.copy_(host_w[i], non_blocking=True)
-            st = wl.L.mx_quantize(*wl.quant_calls[i], ctypes.c_void_p(sp))
-            assert st == 0
-            for j in (2 * i, 2 * i + 1):
-                st = wl.L.mx_grid_equal(*wl.cmp_calls[j], ctypes.c_void_p(sp))
-                assert st == 0
+        wl.quantize_all(ctypes.c_void_p(sp))
+        wl.compare_all(ctypes.c_void_p(sp))
+        for i, (W, q, s, qs, ss) in enumerate(wl.items):
             host_q[i].copy_(q, non_blocking=True)
             host_s[i].copy_(s, non_blocking=True)
         host_r.copy_(wl.results, non_blocking=True)
@@ -362,7 +363,7 @@ def run_e2e(wl, args, device):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    ok = int(host_r[:, :, 0].sum()) == 0
+    ok = int(host_r[0].sum()) == 0
     del host_w, host_q, host_s
     return {"value": round(wl.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 2), "steps": steps, "grid_equal": ok}
@@ -467,8 +468,69 @@ def run_secondary(device, peaks, reps=10):
     return out
 
 
+CASES = ("quant-gate-up", "quant-dy-rowcol", "gemm-fwd-10300", "gemm-update-fprop", "gemm-moe-gate-up",
+         "gemm-moe-down", "grid-equal-gate-up")
+
+
+def run_case(name: str, reps: int):
+    """One kernel on one config, `reps` launches, for profiler captures (prints its CUDA-event time)."""
+    import torch
+
+    from mxfp8_block_scaled_07_b200 import build as mxbuild
+    from mxfp8_block_scaled_07_b200 import mx, synth
+
+    mxbuild.build()
+    dev = torch.device("cuda", 0)
+    if name == "quant-gate-up":
+        x = synth.sync_weight(0, 2, device=dev)
+        bufs = mx.quantize(x, True, False)
+        fn = lambda: mx.quantize(x, True, False, out=bufs)
+    elif name == "quant-dy-rowcol":
+        _, _, x = synth.update_inputs(device=dev)
+        bufs = mx.quantize(x, True, True)
+        fn = lambda: mx.quantize(x, True, True, out=bufs)
+    elif name == "grid-equal-gate-up":
+        x = synth.sync_weight(0, 2, device=dev)
+        q, _, _, _ = mx.quantize(x, True, False)
+        q2 = q.clone()
+        fn = lambda: mx.grid_equal(q, q2)
+    elif name.startswith("gemm-moe"):
+        counts, Xp, Hh, W1, W2 = synth.moe_inputs(device=dev)
+        counts = [int(c) for c in counts]
+        A, Wt = (Xp, W1) if name == "gemm-moe-gate-up" else (Hh, W2)
+        G, N, K = Wt.shape
+        qa, sa_raw, _, _ = mx.quantize(A, True, False, swizzle=False)
+        sa = mx.swizzle_scales(sa_raw, counts)
+        qb, sb, _, _ = mx.quantize(Wt.reshape(G * N, K), True, False)
+        offs = torch.tensor(synth.group_offsets(counts), dtype=torch.int32, device=dev)
+        C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: mx.grouped_gemm(qa, sa, qb.reshape(G, N, K), sb, offs, out=C)
+    else:
+        if name == "gemm-fwd-10300":
+            A = synth.fwd_activations(10300, device=dev)
+            B = synth.sync_weight(0, 2, device=dev)
+        else:
+            A, B, _ = synth.update_inputs(device=dev)
+        qa, sa, _, _ = mx.quantize(A, True, False)
+        qb, sb, _, _ = mx.quantize(B, True, False)
+        C = torch.empty((A.shape[0], B.shape[0]), dtype=torch.bfloat16, device=dev)
+        fn = lambda: mx.gemm(qa, sa, qb, sb, out=C)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, "reps": reps, "ms_per_launch": e0.elapsed_time(e1) / reps,
+                      "device_error": mx.device_error()}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=CASES, help="run one kernel config only (for profiler captures)")
+    ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -477,6 +539,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args.case, args.reps)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
@@ -519,18 +583,18 @@ def main():
     quant_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
     cmp_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
     ms = max_over_ranks(pg, ms_local)
-    mismatches = sum_over_ranks(pg, int(wl.results[:, :, 0].sum().item()))
+    mismatches = sum_over_ranks(pg, int(wl.results[0].sum().item()))
     value = world * wl.step_bytes / (ms * 1e-3) / 1e9
 
-    quant_launch_ms = quant_ms / len(wl.quant_calls)
-    quant_bytes_per_launch = wl.quant_bytes / len(wl.quant_calls)
+    quant_launch_ms = quant_ms          # one mx_quantize_multi launch per step
+    quant_bytes_per_launch = wl.quant_bytes
     achieved = quant_bytes_per_launch / (quant_launch_ms * 1e-3) / 1e9
     trec = traffic_record()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": (round(trec["dram_bytes_per_elem"] * wl.total_elems / len(wl.quant_calls))
+                "traffic": (round(trec["dram_bytes_per_elem"] * wl.total_elems)
                             if trec else None),
-                "kernel": "quantize_kernel<rowwise> (mx_quantize ROWWISE|SWIZZLE)",
+                "kernel": "quantize_kernel<rowwise, multi-tensor> (mx_quantize_multi ROWWISE|SWIZZLE, 144 tensors)",
                 "peak_source": f"{peaks['source']} hbm copy (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
                 else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": round(quant_bytes_per_launch),
@@ -564,7 +628,7 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * (144 + 2 * 288),
+            "gpu_launches": args.steps * SyncWorkload.LAUNCHES_PER_STEP,
             "clocks": clocks.summary(),
             "grid_equal_mismatches": mismatches,
             "secondary": secondary,

@@ -83,6 +83,26 @@ mx_status mx_quantize(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, in
                       uint8_t* q_row, uint8_t* s_row, uint8_t* q_col, uint8_t* s_col,
                       mx_stream stream);
 
+/* One tensor of a multi-tensor quantization: the arguments of mx_quantize, same meaning. */
+typedef struct {
+    const void* x;            /* BF16 [M, K], row stride ld_x elements (device) */
+    int64_t M, K, ld_x;
+    uint8_t* q_row;           /* outputs of the requested directions (device) */
+    uint8_t* s_row;
+    uint8_t* q_col;
+    uint8_t* s_col;
+} mx_quant_tensor;
+
+/*
+ * mx_quantize over a list of tensors with the same flags, in as few launches as possible (one per
+ * 192 tensors). At every weight synchronization the learner quantizes every weight of the model
+ * (Figure 1); walking all tensors' tiles as one tile space removes the per-launch ramp and tail.
+ * `tensors` is host memory, read during the call. Every tensor is checked as by mx_quantize before
+ * anything is launched; the first failing check's status is returned. Results are identical to
+ * one mx_quantize call per tensor. Outputs of different tensors must not overlap.
+ */
+mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags, mx_stream stream);
+
 /*
  * Scale rearrangement (Table 6, "scale rearrangement"; Table 10 F3, the interleaved scale copy a
  * backend derives): raw scales s[rows, kblocks] (device, packed) -> the tensor-core layout in
@@ -143,6 +163,22 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
 mx_status mx_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes,
                         unsigned long long* mismatches_dev, long long* first_index_dev,
                         mx_stream stream);
+
+/* One pair of a multi-pair byte comparison. */
+typedef struct {
+    const uint8_t* a;         /* device */
+    const uint8_t* b;         /* device */
+    int64_t nbytes;
+} mx_compare_pair;
+
+/*
+ * mx_grid_equal over n pairs in one pass (the byte comparison of a whole synchronization: every
+ * weight's elements, raw scales and swizzled scales). For pair i, mismatches_dev[i] (uint64) and
+ * first_index_dev[i] (int64, -1 if equal) are written (device arrays of n entries each). `pairs`
+ * is host memory, read during the call. Results are identical to n mx_grid_equal calls.
+ */
+mx_status mx_grid_equal_multi(const mx_compare_pair* pairs, int64_t n, unsigned long long* mismatches_dev,
+                              long long* first_index_dev, mx_stream stream);
 
 /* Human-readable name of a status code (static string). */
 const char* mx_status_string(mx_status status);

@@ -15,6 +15,7 @@
 #include "grid_equal.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
+#include "swizzle.cuh"
 
 namespace mx {
 
@@ -45,7 +46,7 @@ struct DeviceInfo {
     int cc_major = 0;
     uint32_t* status = nullptr;
     int quant_blocks_per_sm[4] = {0, 0, 0, 0};
-    bool gemm_attr_set = false;
+    int ge_blocks_per_sm = 1;
     bool ok = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -60,7 +61,7 @@ std::once_flag g_encode_once;
 template <bool R, bool C>
 int quant_occupancy() {
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<R, C>, kQThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<R, C, kQMaxTensors>, kQThreads, 0);
     return n > 0 ? n : 1;
 }
 
@@ -81,9 +82,14 @@ const DeviceInfo* device_info() {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
         d.status = static_cast<uint32_t*>(p);
-        d.quant_blocks_per_sm[1] = quant_occupancy<true, false>();
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1], quantize_rowwise_kernel<kQMaxTensors>,
+                                                      kQThreads, 0);
+        if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
         d.quant_blocks_per_sm[2] = quant_occupancy<false, true>();
         d.quant_blocks_per_sm[3] = quant_occupancy<true, true>();
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.ge_blocks_per_sm, grid_equal_kernel<kGeMaxPairs>,
+                                                      kGeThreads, 0);
+        if (d.ge_blocks_per_sm < 1) d.ge_blocks_per_sm = 1;
         if (cudaFuncSetAttribute(mx_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemDense) != cudaSuccess ||
             cudaFuncSetAttribute(mx_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -197,45 +203,128 @@ mx_status mx_diag_expired_wait(mx_stream stream) {
     return launched();
 }
 
+}  // extern "C"
+
+namespace mx {
+namespace {
+
+// Validates one tensor of a quantize call; *empty is set when it has no elements.
+mx_status check_quant_tensor(const mx_quant_tensor& t, bool row, bool col, bool* empty) {
+    if (t.M < 0 || t.K < 0) return MX_ERR_ARG;
+    if (t.K % 32 != 0 || (col && t.M % 32 != 0)) return MX_ERR_SHAPE;
+    *empty = (t.M == 0 || t.K == 0);
+    if (*empty) return MX_OK;   // empty tensors may carry null pointers
+    if (!t.x || (row && (!t.q_row || !t.s_row)) || (col && (!t.q_col || !t.s_col))) return MX_ERR_ARG;
+    if (t.ld_x < t.K) return MX_ERR_SHAPE;
+    if (!aligned16(t.x) || t.ld_x % 8 != 0) return MX_ERR_ALIGN;
+    if (row && (!aligned16(t.q_row) || !aligned16(t.s_row))) return MX_ERR_ALIGN;
+    if (col && (!aligned16(t.q_col) || !aligned16(t.s_col))) return MX_ERR_ALIGN;
+    return MX_OK;
+}
+
+template <int NT>
+void add_quant_tensor(QuantArgs<NT>& a, const mx_quant_tensor& t) {
+    QTensor& q = a.t[a.n++];
+    q.x = static_cast<const uint16_t*>(t.x);
+    q.q_row = t.q_row;
+    q.s_row = t.s_row;
+    q.q_col = t.q_col;
+    q.s_col = t.s_col;
+    q.M = t.M;
+    q.K = t.K;
+    q.ldx = t.ld_x;
+    q.tiles_m = static_cast<int32_t>(ceil_div(t.M, kQTile));
+    q.tiles_k = static_cast<int32_t>(ceil_div(t.K, kQTile));
+    q.vec32 = (reinterpret_cast<uintptr_t>(t.x) % 32 == 0) && (t.ld_x % 16 == 0) &&
+              (reinterpret_cast<uintptr_t>(t.q_row) % 32 == 0);
+    q.tile_start = a.total_tiles;
+    a.total_tiles += int64_t(q.tiles_m) * q.tiles_k;
+}
+
+template <int NT>
+mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceInfo* d, mx_stream stream) {
+    if (a.total_tiles == 0) return MX_OK;
+    const int which = (row ? 1 : 0) | (col ? 2 : 0);
+    const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
+    if (row && col)
+        quantize_kernel<true, true, NT><<<grid, kQThreads, 0, stream>>>(a);
+    else if (row)
+        quantize_rowwise_kernel<NT><<<grid, kQThreads, 0, stream>>>(a);
+    else
+        quantize_kernel<false, true, NT><<<grid, kQThreads, 0, stream>>>(a);
+    return launched();
+}
+
+template <int NP>
+void add_pair(CmpArgs<NP>& g, const uint8_t* a, const uint8_t* b, int64_t nbytes) {
+    CmpPair& p = g.p[g.n++];
+    p.a = a;
+    p.b = b;
+    p.nbytes = nbytes;
+    p.vec = aligned16(a) && aligned16(b);
+    p.unit_start = g.total_units;
+    g.total_units += ceil_div(nbytes, kGeUnitBytes);
+}
+
+template <int NP>
+mx_status launch_compare(const CmpArgs<NP>& g, const DeviceInfo* d, mx_stream stream) {
+    grid_equal_reset_kernel<<<static_cast<int>(ceil_div(g.n, 256)), 256, 0, stream>>>(g.counts, g.firsts, g.n);
+    if (mx_status st = launched()) return st;
+    if (g.total_units == 0) return MX_OK;
+    const int64_t grid = std::min<int64_t>(g.total_units, int64_t(d->sms) * d->ge_blocks_per_sm);
+    grid_equal_kernel<NP><<<grid, kGeThreads, 0, stream>>>(g);
+    return launched();
+}
+
+}  // namespace
+}  // namespace mx
+
+extern "C" {
+
 mx_status mx_quantize(const void* x, int64_t M, int64_t K, int64_t ld_x, int flags, uint8_t* q_row,
                       uint8_t* s_row, uint8_t* q_col, uint8_t* s_col, mx_stream stream) {
     const bool row = flags & MX_ROWWISE, col = flags & MX_COLWISE, swz = flags & MX_SWIZZLE;
     if (flags & ~(MX_ROWWISE | MX_COLWISE | MX_SWIZZLE)) return MX_ERR_ARG;
     if (!row && !col) return MX_ERR_ARG;
-    if (M < 0 || K < 0) return MX_ERR_ARG;
-    if (K % 32 != 0 || (col && M % 32 != 0)) return MX_ERR_SHAPE;
-    if (M == 0 || K == 0) return MX_OK;   // empty tensors may carry null pointers
-    if (!x || (row && (!q_row || !s_row)) || (col && (!q_col || !s_col))) return MX_ERR_ARG;
-    if (ld_x < K) return MX_ERR_SHAPE;
-    if (!aligned16(x) || ld_x % 8 != 0) return MX_ERR_ALIGN;
-    if (row && (!aligned16(q_row) || !aligned16(s_row))) return MX_ERR_ALIGN;
-    if (col && (!aligned16(q_col) || !aligned16(s_col))) return MX_ERR_ALIGN;
+    const mx_quant_tensor t{x, M, K, ld_x, q_row, s_row, q_col, s_col};
+    bool empty = false;
+    if (mx_status st = check_quant_tensor(t, row, col, &empty)) return st;
+    if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
+    QuantArgs<1> a;
+    a.n = 0;
+    a.swz = swz;
+    a.total_tiles = 0;
+    add_quant_tensor(a, t);
+    return launch_quant(a, row, col, d, stream);
+}
 
-    QuantArgs a;
-    a.x = static_cast<const uint16_t*>(x);
-    a.M = M;
-    a.K = K;
-    a.ldx = ld_x;
-    a.q_row = q_row;
-    a.s_row = s_row;
-    a.q_col = q_col;
-    a.s_col = s_col;
-    a.swz_row = swz;
-    a.swz_col = swz;
-    a.tiles_m = ceil_div(M, kQTile);
-    a.tiles_k = ceil_div(K, kQTile);
-    a.tiles = a.tiles_m * a.tiles_k;
-    const int which = (row ? 1 : 0) | (col ? 2 : 0);
-    const int64_t grid = std::min<int64_t>(a.tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
-    if (row && col)
-        quantize_kernel<true, true><<<grid, kQThreads, 0, stream>>>(a);
-    else if (row)
-        quantize_kernel<true, false><<<grid, kQThreads, 0, stream>>>(a);
-    else
-        quantize_kernel<false, true><<<grid, kQThreads, 0, stream>>>(a);
-    return launched();
+mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags, mx_stream stream) {
+    const bool row = flags & MX_ROWWISE, col = flags & MX_COLWISE, swz = flags & MX_SWIZZLE;
+    if (flags & ~(MX_ROWWISE | MX_COLWISE | MX_SWIZZLE)) return MX_ERR_ARG;
+    if (!row && !col) return MX_ERR_ARG;
+    if (n < 0 || (n > 0 && !tensors)) return MX_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        bool empty = false;
+        if (mx_status st = check_quant_tensor(tensors[i], row, col, &empty)) return st;
+    }
+    if (n == 0) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    static thread_local QuantArgs<kQMaxTensors> a;   // ~14 KB: kept off the stack
+    for (int64_t i0 = 0; i0 < n; i0 += kQMaxTensors) {
+        a.n = 0;
+        a.swz = swz;
+        a.total_tiles = 0;
+        for (int64_t i = i0; i < std::min<int64_t>(n, i0 + kQMaxTensors); ++i) {
+            const mx_quant_tensor& t = tensors[i];
+            if (t.M > 0 && t.K > 0) add_quant_tensor(a, t);
+        }
+        if (a.n == 0) continue;
+        if (mx_status st = launch_quant(a, row, col, d, stream)) return st;
+    }
+    return MX_OK;
 }
 
 mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, const int64_t* group_rows_host,
@@ -292,14 +381,34 @@ mx_status mx_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes, unsi
     if (!mismatches_dev || !first_index_dev || nbytes < 0 || (nbytes > 0 && (!a || !b))) return MX_ERR_ARG;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    grid_equal_reset_kernel<<<1, 1, 0, stream>>>(mismatches_dev, first_index_dev);
-    if (mx_status st = launched()) return st;
-    if (nbytes == 0) return MX_OK;
-    const int vec = aligned16(a) && aligned16(b);
-    const int64_t work = vec ? ceil_div(nbytes, 16 * kGeUnroll) : nbytes;
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(work, kGeThreads), int64_t(d->sms) * 8));
-    grid_equal_kernel<<<grid, kGeThreads, 0, stream>>>(a, b, nbytes, vec, mismatches_dev, first_index_dev);
-    return launched();
+    CmpArgs<1> g;
+    g.n = 0;
+    g.total_units = 0;
+    g.counts = mismatches_dev;
+    g.firsts = first_index_dev;
+    add_pair(g, a, b, nbytes);
+    return launch_compare(g, d, stream);
+}
+
+mx_status mx_grid_equal_multi(const mx_compare_pair* pairs, int64_t n, unsigned long long* mismatches_dev,
+                              long long* first_index_dev, mx_stream stream) {
+    if (n < 0 || (n > 0 && (!pairs || !mismatches_dev || !first_index_dev))) return MX_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        if (pairs[i].nbytes < 0 || (pairs[i].nbytes > 0 && (!pairs[i].a || !pairs[i].b))) return MX_ERR_ARG;
+    if (n == 0) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    static thread_local CmpArgs<kGeMaxPairs> g;      // ~20 KB: kept off the stack
+    for (int64_t i0 = 0; i0 < n; i0 += kGeMaxPairs) {
+        g.n = 0;
+        g.total_units = 0;
+        g.counts = mismatches_dev + i0;
+        g.firsts = first_index_dev + i0;
+        for (int64_t i = i0; i < std::min<int64_t>(n, i0 + kGeMaxPairs); ++i)
+            add_pair(g, pairs[i].a, pairs[i].b, pairs[i].nbytes);
+        if (mx_status st = launch_compare(g, d, stream)) return st;
+    }
+    return MX_OK;
 }
 
 mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz, int64_t M,

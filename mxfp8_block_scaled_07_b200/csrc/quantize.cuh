@@ -1,19 +1,21 @@
-// MXFP8 quantizer (rowwise and/or columnwise, optionally writing the tensor-core scale layout
-// directly) and the standalone scale rearrangement.
+// MXFP8 quantizer: rowwise and/or columnwise, optionally writing the tensor-core scale layout
+// directly, over one tensor or a list of tensors in one launch.
 //
 // The paper ("End-to-End MXFP8 Reinforcement Learning on Blackwell", Figure 1 and Table 6) has the
-// learner quantize BF16 masters and activations, then rearrange the E8M0 scales ("scale
+// learner quantize BF16 masters and activations and then rearrange the E8M0 scales ("scale
 // rearrangement", 2.6 ms per micro-batch, more than the 2.2 ms of quantization). Here both happen in
-// one HBM pass: a CTA owns a 128 x 128 BF16 tile, whose rowwise scales (128 rows x 4 K-blocks) and
-// columnwise scales (128 K-rows x 4 M-blocks) are each exactly one 512-byte block of the
-// tensor-core scale layout, so the swizzled scales leave the CTA as one coalesced 512-byte store.
+// one HBM pass: a CTA iteration owns a 128 x 128 BF16 tile, whose rowwise scales (128 rows x 4
+// K-blocks) and columnwise scales (128 K-rows x 4 M-blocks) are each exactly one 512-byte block of
+// the tensor-core scale layout, so the swizzled scales leave the CTA as one coalesced 512-byte store.
+// At weight synchronization every weight of the model is quantized (Figure 1); the multi-tensor
+// form walks the tiles of all of them as one tile space, so one persistent launch covers the model.
 //
-// Rule (OCP MX v1.0, which the paper's "E8M0 scales keep only the exponent", Table 10 F6, refers
-// to): per 32-block, e = floor(log2 amax) - 8 clamped to [-127, 127], scale byte e + 127;
-// elements RNE(x * 2^-e) saturated to +-448 in E4M3. For BF16 input, floor(log2 amax) is the
-// biased exponent field minus 127, so the scale byte is max(E_amax - 8, 0), computed on integer
-// bits. x * 2^-e is exact in fp32, and one cvt.rn.satfinite rounds it. Blocks holding NaN or Inf
-// get scale 0xFF and element bytes sign|0x7F.
+// Rule (OCP MX v1.0; the paper's "E8M0 scales keep only the exponent", Table 10 F6): per 32-block,
+// e = floor(log2 amax) - 8 clamped to [-127, 127], scale byte e + 127; elements RNE(x * 2^-e)
+// saturated to +-448 in E4M3. For BF16 input floor(log2 amax) is the biased exponent field minus
+// 127, so the scale byte is max(E_amax - 8, 0), computed on integer bits. x * 2^-e is exact in fp32
+// (a packed fp32x2 multiply) and one cvt.rn.satfinite rounds it. Blocks holding NaN or Inf get
+// scale 0xFF and element bytes sign|0x7F.
 //
 // This file must not be compiled with flush-to-zero: BF16 subnormal inputs scaled by 2^127 are
 // normal E4M3 values.
@@ -26,6 +28,7 @@ namespace mx {
 
 constexpr int kQTile = 128;          // rows and columns of a quantizer tile
 constexpr int kQThreads = 256;
+constexpr int kQMaxTensors = 192;    // tensors per multi-tensor launch (kernel parameters < 32 KB)
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     uint4 v;
@@ -35,17 +38,18 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
+// max(|a|, |b|) per BF16 half, NaN-propagating (a NaN operand gives the canonical NaN 0x7FFF);
+// the sign bits of the result are garbage and are masked by the caller.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
-}
-
-// Packs RNE-saturated E4M3 codes of (hi, lo) into 16 bits: lo in bits 0-7, hi in bits 8-15.
-__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
 }
 
 // Scale byte from the largest BF16 magnitude bits of a block (0 .. 0x7FFF).
@@ -55,33 +59,164 @@ __device__ __forceinline__ uint32_t scale_byte_from_amax(uint32_t amax_bits) {
     return static_cast<uint32_t>(E > 8 ? E - 8 : 0);
 }
 
-// 2^-e as an fp32 for scale byte s = e + 127 (s <= 246 for BF16 input): biased exponent 254 - s.
-__device__ __forceinline__ float inv_scale(uint32_t s) {
-    return s <= 246u ? __uint_as_float((254u - s) << 23) : 1.0f;
+// {2^-e, 2^-e} as a packed fp32 pair for scale byte s = e + 127 <= 246: biased exponent 254 - s.
+__device__ __forceinline__ uint64_t inv_scale2(uint32_t s) {
+    const uint32_t f = (254u - s) << 23;
+    return (static_cast<uint64_t>(f) << 32) | f;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Two BF16 (one word) -> two E4M3 codes (16 bits), given the block's scale byte and 2^-e.
-__device__ __forceinline__ uint32_t encode_word(uint32_t w, uint32_t s, float inv) {
-    if (s == 0xFFu) return 0x7F7Fu | ((w >> 8) & 0x80u) | (((w >> 24) & 0x80u) << 8);
-    return cvt_e4m3x2(bf16_hi(w) * inv, bf16_lo(w) * inv);
+// E4M3 codes of four values given as fp32 bit patterns (e0 -> bits 0-7 ... e3 -> bits 24-31),
+// after scaling all by the packed pair inv2.
+__device__ __forceinline__ uint32_t enc_quad(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3, uint64_t inv2) {
+    uint32_t r;
+    asm("{\n\t.reg .b64 x0, x1, y0, y1;\n\t.reg .b32 l0, h0, l1, h1;\n\t.reg .b16 c0, c1;\n\t"
+        "mov.b64 x0, {%1, %2};\n\t"
+        "mov.b64 x1, {%3, %4};\n\t"
+        "mul.rn.f32x2 y0, x0, %5;\n\t"
+        "mul.rn.f32x2 y1, x1, %5;\n\t"
+        "mov.b64 {l0, h0}, y0;\n\t"
+        "mov.b64 {l1, h1}, y1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c0, h0, l0;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c1, h1, l1;\n\t"
+        "mov.b32 %0, {c0, c1};\n\t}"
+        : "=r"(r)
+        : "r"(e0), "r"(e1), "r"(e2), "r"(e3), "l"(inv2));
+    return r;
 }
 
-struct QuantArgs {
+// Four BF16 (two words, element 0 in the low half of w0) -> four E4M3 bytes (element 0 in bits
+// 0-7), scaled by the packed pair inv2.
+__device__ __forceinline__ uint32_t enc_words(uint32_t w0, uint32_t w1, uint64_t inv2) {
+    uint32_t r;
+    asm("{\n\t.reg .b64 x0, x1, y0, y1;\n\t.reg .b32 l0, h0, l1, h1;\n\t.reg .b16 c0, c1;\n\t"
+        "shl.b32 l0, %1, 16;\n\t"
+        "and.b32 h0, %1, 0xFFFF0000;\n\t"
+        "shl.b32 l1, %2, 16;\n\t"
+        "and.b32 h1, %2, 0xFFFF0000;\n\t"
+        "mov.b64 x0, {l0, h0};\n\t"
+        "mov.b64 x1, {l1, h1};\n\t"
+        "mul.rn.f32x2 y0, x0, %3;\n\t"
+        "mul.rn.f32x2 y1, x1, %3;\n\t"
+        "mov.b64 {l0, h0}, y0;\n\t"
+        "mov.b64 {l1, h1}, y1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c0, h0, l0;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c1, h1, l1;\n\t"
+        "mov.b32 %0, {c0, c1};\n\t}"
+        : "=r"(r)
+        : "r"(w0), "r"(w1), "l"(inv2));
+    return r;
+}
+
+// Eight BF16 (one 16-byte chunk, element 0 in the low half of v.x) -> eight E4M3 bytes.
+__device__ __forceinline__ uint2 encode_chunk(const uint4 v, uint32_t s) {
+    uint2 o;
+    if (s != 0xFFu) {
+        const uint64_t inv2 = inv_scale2(s);
+        o.x = enc_words(v.x, v.y, inv2);
+        o.y = enc_words(v.z, v.w, inv2);
+    } else {
+        // NaN/Inf block: every element byte is sign | 0x7F.
+        const uint32_t m = 0x7F7F7F7Fu;
+        o.x = m | ((v.x >> 8) & 0x80u) | ((v.x >> 16) & 0x8000u) | ((v.y << 8) & 0x800000u) | (v.y & 0x80000000u);
+        o.y = m | ((v.z >> 8) & 0x80u) | ((v.z >> 16) & 0x8000u) | ((v.w << 8) & 0x800000u) | (v.w & 0x80000000u);
+    }
+    return o;
+}
+
+struct QTensor {
     const uint16_t* x;
-    int64_t M, K, ldx;
     uint8_t* q_row;
     uint8_t* s_row;
     uint8_t* q_col;
     uint8_t* s_col;
-    int swz_row, swz_col;
-    int64_t tiles_m, tiles_k, tiles;
+    int64_t M, K, ldx;
+    int64_t tile_start;       // first tile of this tensor in the launch's tile space
+    int32_t tiles_m, tiles_k;
+    int32_t vec32;            // x rows and q_row 32-byte aligned: 256-bit loads and stores
 };
 
-template <bool ROW, bool COL>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) {
+struct Block32 {
+    uint4 v[4];               // 32 BF16, element 0 in the low half of v[0].x
+};
+
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint4& a, uint4& b) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
+__device__ __forceinline__ uint4 ld_cached_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v8(void* p, const uint4& a, const uint4& b) {
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y),
+                 "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
+template <int NT>
+struct QuantArgs {
+    int n;                    // tensors in this launch
+    int swz;                  // write the tensor-core scale layout (else raw scales)
+    int64_t total_tiles;
+    QTensor t[NT];
+};
+
+struct TileRef {
+    int i;                    // tensor index
+    int64_t m0, k0;
+    int mt, kt;
+    bool full;                // the whole 128 x 128 tile lies inside the tensor
+};
+
+template <int NT>
+__device__ __forceinline__ TileRef decode_qtile(const QuantArgs<NT>& a, int64_t t) {
+    int i = 0;
+    if constexpr (NT > 1) {
+        int lo = 0, hi = a.n - 1;    // largest i with tile_start <= t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.t[mid].tile_start <= t) lo = mid; else hi = mid - 1;
+        }
+        i = lo;
+    }
+    const QTensor& T = a.t[i];
+    const int64_t local = t - T.tile_start;
+    TileRef r;
+    r.i = i;
+    r.mt = static_cast<int>(local / T.tiles_k);
+    r.kt = static_cast<int>(local % T.tiles_k);
+    r.m0 = static_cast<int64_t>(r.mt) * kQTile;
+    r.k0 = static_cast<int64_t>(r.kt) * kQTile;
+    r.full = (r.m0 + kQTile <= T.M) && (r.k0 + kQTile <= T.K);
+    return r;
+}
+
+// Thread tid loads chunk (tid & 15) of rows it * 16 + (tid >> 4), it = 0..7.
+template <int NT>
+__device__ __forceinline__ void load_qtile(const QuantArgs<NT>& a, const TileRef& r, uint4 (&v)[8], int tid) {
+    const QTensor& T = a.t[r.i];
+    const int cc = tid & 15;
+    const uint16_t* base = T.x + (r.m0 + (tid >> 4)) * T.ldx + r.k0 + cc * 8;
+    const int64_t step = 16 * T.ldx;
+    if (r.full) {
+#pragma unroll
+        for (int it = 0; it < 8; ++it) v[it] = ld_stream_v4(base + it * step);
+    } else {
+        const bool kok = r.k0 + cc * 8 < T.K;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const bool ok = kok && (r.m0 + it * 16 + (tid >> 4) < T.M);
+            v[it] = ok ? ld_stream_v4(base + it * step) : make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+template <bool ROW, bool COL, int NT>
+__global__ void __launch_bounds__(kQThreads, 3) quantize_kernel(const __grid_constant__ QuantArgs<NT> a) {
     __shared__ __align__(16) uint4 tile[COL ? kQTile * 16 : 1];   // 128 rows x 16 chunks of 8 BF16
     __shared__ __align__(16) uint8_t atom_row[512];
     __shared__ __align__(16) uint8_t atom_col[512];
@@ -89,30 +224,36 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int64_t kblocks = a.K / 32;
 
+    // Each CTA owns a contiguous range of the tile space: one decode at the start, then the next
+    // tile is found by stepping (tensor, row tile, column tile) without divisions.
+    const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
+    const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
+    const int64_t t_end = min(a.total_tiles, t_begin + per);
     uint4 cur[8], nxt[8];
-    auto load_tile = [&](uint4 (&v)[8], int64_t t) {
-        const int64_t m0 = (t / a.tiles_k) * kQTile, k0 = (t % a.tiles_k) * kQTile;
-        const int cc = tid & 15;
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int row = it * 16 + (tid >> 4);
-            const int64_t m = m0 + row, k = k0 + cc * 8;
-            if (m < a.M && k < a.K)
-                v[it] = ld_stream_v4(a.x + m * a.ldx + k);
-            else
-                v[it] = make_uint4(0, 0, 0, 0);
+    TileRef rc, rn;
+    if (t_begin < t_end) {
+        rc = decode_qtile(a, t_begin);
+        load_qtile(a, rc, cur, tid);
+    }
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        if (t + 1 < t_end) {
+            rn = rc;
+            if (++rn.kt == a.t[rn.i].tiles_k) {
+                rn.kt = 0;
+                if (++rn.mt == a.t[rn.i].tiles_m) {
+                    rn.mt = 0;
+                    ++rn.i;
+                }
+            }
+            const QTensor& Tn = a.t[rn.i];
+            rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
+            rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
+            rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
+            load_qtile(a, rn, nxt, tid);
         }
-    };
-
-    int64_t t = blockIdx.x;
-    if (t < a.tiles) load_tile(cur, t);
-    for (; t < a.tiles; t += gridDim.x) {
-        const int64_t tn = t + gridDim.x;
-        if (tn < a.tiles) load_tile(nxt, tn);
-        const int64_t mt = t / a.tiles_k, kt = t % a.tiles_k;
-        const int64_t m0 = mt * kQTile, k0 = kt * kQTile;
+        const QTensor& T = a.t[rc.i];
+        const int64_t kblocks = T.K / 32;
 
         if constexpr (COL) {
 #pragma unroll
@@ -122,25 +263,19 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) 
         if constexpr (ROW) {
             // Four consecutive lanes hold one 32-block (8 BF16 each) of one row.
             const int cc = tid & 15;
+            const bool kok = rc.k0 + cc * 8 < T.K;
+            uint8_t* qbase = T.q_row + (rc.m0 + (tid >> 4)) * T.K + rc.k0 + cc * 8;
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
                 const int row = it * 16 + (tid >> 4);
-                const int64_t m = m0 + row, k = k0 + cc * 8;
-                const bool valid = (m < a.M) && (k < a.K);
+                const bool valid = rc.full || (kok && rc.m0 + row < T.M);
                 const uint4 v = cur[it];
-                uint32_t mx = max_u16x2(max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                        max_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+                uint32_t mx = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)) & 0x7FFF7FFFu;
                 mx = max(mx & 0xFFFFu, mx >> 16);
                 mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
                 mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
                 const uint32_t s = scale_byte_from_amax(mx);
-                const float inv = inv_scale(s);
-                if (valid) {
-                    uint2 o;
-                    o.x = encode_word(v.x, s, inv) | (encode_word(v.y, s, inv) << 16);
-                    o.y = encode_word(v.z, s, inv) | (encode_word(v.w, s, inv) << 16);
-                    *reinterpret_cast<uint2*>(a.q_row + m * a.K + k) = o;
-                }
+                if (valid) *reinterpret_cast<uint2*>(qbase + it * 16 * T.K) = encode_chunk(v, s);
                 if ((lane & 3) == 0)
                     atom_row[(row & 31) * 16 + (row >> 5) * 4 + (cc >> 2)] = valid ? static_cast<uint8_t>(s) : 0;
             }
@@ -149,7 +284,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) 
         if constexpr (COL) {
             __syncthreads();
             // Warp w: M-block (w >> 1) of 32 rows, chunks (w & 1) * 8 .. +7; lane = chunk (low 3
-            // bits) + 8 * (8-row group inside the M-block). Each lane reads 8 rows x 8 columns.
+            // bits) + 8 * (8-row group inside the M-block). Each lane owns 8 rows x 8 columns.
             const int chunk = (warp & 1) * 8 + (lane & 7);
             const int rgq = lane >> 3;
             const int mb = warp >> 1;
@@ -163,40 +298,40 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) 
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t word = (w == 0 ? r[i].x : w == 1 ? r[i].y : w == 2 ? r[i].z : r[i].w);
-                    mm = max_u16x2(mm, word & 0x7FFF7FFFu);
+                    mm = bf16x2_absmax(mm, word);
                 }
+                mm &= 0x7FFF7FFFu;
                 mm = max_u16x2(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 8));
                 mm = max_u16x2(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 16));
                 m4[w] = mm;
             }
-            const int64_t kcol0 = k0 + chunk * 8;
-            const int64_t mrow0 = m0 + mb * 32;
-            const bool valid = (kcol0 < a.K) && (mrow0 < a.M);
+            const int64_t kcol0 = rc.k0 + chunk * 8;
+            const int64_t mrow0 = rc.m0 + mb * 32;
+            const bool valid = rc.full || ((kcol0 < T.K) && (mrow0 < T.M));
+            uint8_t* qbase = T.q_col + kcol0 * T.M + mrow0 + rgq * 8;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int w = j >> 1, h = j & 1;
                 const uint32_t amax = h ? (m4[w] >> 16) : (m4[w] & 0xFFFFu);
                 const uint32_t s = scale_byte_from_amax(amax);
-                const float inv = inv_scale(s);
-                uint32_t e[8];
+                uint32_t e[8];       // (row i, column j) widened to fp32 bits
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t word = (w == 0 ? r[i].x : w == 1 ? r[i].y : w == 2 ? r[i].z : r[i].w);
-                    e[i] = h ? (word >> 16) : (word & 0xFFFFu);      // BF16 bits of (row i, column j)
+                    e[i] = h ? (word & 0xFFFF0000u) : (word << 16);
                 }
                 uint2 o;
-                if (s == 0xFFu) {
-                    o.x = 0x7F7F7F7Fu | ((e[0] >> 8) & 0x80u) | (((e[1] >> 8) & 0x80u) << 8) |
-                          (((e[2] >> 8) & 0x80u) << 16) | (((e[3] >> 8) & 0x80u) << 24);
-                    o.y = 0x7F7F7F7Fu | ((e[4] >> 8) & 0x80u) | (((e[5] >> 8) & 0x80u) << 8) |
-                          (((e[6] >> 8) & 0x80u) << 16) | (((e[7] >> 8) & 0x80u) << 24);
+                if (s != 0xFFu) {
+                    const uint64_t inv2 = inv_scale2(s);
+                    o.x = enc_quad(e[0], e[1], e[2], e[3], inv2);
+                    o.y = enc_quad(e[4], e[5], e[6], e[7], inv2);
                 } else {
-                    o.x = cvt_e4m3x2(__uint_as_float(e[1] << 16) * inv, __uint_as_float(e[0] << 16) * inv) |
-                          (cvt_e4m3x2(__uint_as_float(e[3] << 16) * inv, __uint_as_float(e[2] << 16) * inv) << 16);
-                    o.y = cvt_e4m3x2(__uint_as_float(e[5] << 16) * inv, __uint_as_float(e[4] << 16) * inv) |
-                          (cvt_e4m3x2(__uint_as_float(e[7] << 16) * inv, __uint_as_float(e[6] << 16) * inv) << 16);
+                    o.x = 0x7F7F7F7Fu | ((e[0] >> 24) & 0x80u) | ((e[1] >> 16) & 0x8000u) |
+                          ((e[2] >> 8) & 0x800000u) | (e[3] & 0x80000000u);
+                    o.y = 0x7F7F7F7Fu | ((e[4] >> 24) & 0x80u) | ((e[5] >> 16) & 0x8000u) |
+                          ((e[6] >> 8) & 0x800000u) | (e[7] & 0x80000000u);
                 }
-                if (valid) *reinterpret_cast<uint2*>(a.q_col + (kcol0 + j) * a.M + mrow0 + rgq * 8) = o;
+                if (valid) *reinterpret_cast<uint2*>(qbase + j * T.M) = o;
                 if (rgq == 0) {
                     const int kk = chunk * 8 + j;   // K-row inside the tile
                     atom_col[(kk & 31) * 16 + (kk >> 5) * 4 + mb] = valid ? static_cast<uint8_t>(s) : 0;
@@ -207,77 +342,155 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantArgs a) 
         __syncthreads();
         // Scale output: one 512-byte block of the tensor-core layout per direction, or raw bytes.
         if constexpr (ROW) {
-            if (a.swz_row) {
+            if (a.swz) {
                 if (tid < 32)
-                    reinterpret_cast<uint4*>(a.s_row + (mt * a.tiles_k + kt) * 512)[tid] =
+                    reinterpret_cast<uint4*>(T.s_row + (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512)[tid] =
                         reinterpret_cast<const uint4*>(atom_row)[tid];
             } else if (tid < kQTile) {
-                const int64_t m = m0 + tid;
-                const int64_t nb = (kblocks - kt * 4 < 4 ? kblocks - kt * 4 : 4);
-                if (m < a.M)
+                const int64_t m = rc.m0 + tid;
+                const int64_t nb = (kblocks - rc.kt * 4 < 4 ? kblocks - rc.kt * 4 : 4);
+                if (m < T.M)
                     for (int b = 0; b < nb; ++b)
-                        a.s_row[m * kblocks + kt * 4 + b] = atom_row[(tid & 31) * 16 + (tid >> 5) * 4 + b];
+                        T.s_row[m * kblocks + rc.kt * 4 + b] = atom_row[(tid & 31) * 16 + (tid >> 5) * 4 + b];
             }
         }
         if constexpr (COL) {
-            const int64_t mblocks = a.M / 32;
+            const int64_t mblocks = T.M / 32;
             const int u = tid - 128;
-            if (a.swz_col) {
+            if (a.swz) {
                 if (u >= 0 && u < 32)
-                    reinterpret_cast<uint4*>(a.s_col + (kt * a.tiles_m + mt) * 512)[u] =
+                    reinterpret_cast<uint4*>(T.s_col + (static_cast<int64_t>(rc.kt) * T.tiles_m + rc.mt) * 512)[u] =
                         reinterpret_cast<const uint4*>(atom_col)[u];
             } else if (u >= 0) {
-                const int64_t k = k0 + u;
-                const int64_t nb = (mblocks - mt * 4 < 4 ? mblocks - mt * 4 : 4);
-                if (k < a.K)
+                const int64_t k = rc.k0 + u;
+                const int64_t nb = (mblocks - rc.mt * 4 < 4 ? mblocks - rc.mt * 4 : 4);
+                if (k < T.K)
                     for (int b = 0; b < nb; ++b)
-                        a.s_col[k * mblocks + mt * 4 + b] = atom_col[(u & 31) * 16 + (u >> 5) * 4 + b];
+                        T.s_col[k * mblocks + rc.mt * 4 + b] = atom_col[(u & 31) * 16 + (u >> 5) * 4 + b];
             }
         }
         __syncthreads();
 #pragma unroll
         for (int it = 0; it < 8; ++it) cur[it] = nxt[it];
+        rc = rn;
     }
 }
 
-// ---- standalone scale rearrangement ---------------------------------------------------------
+// ---- rowwise-only kernel: one thread per 32-element block ----------------------------------
+//
+// Thread tid owns blocks (row tid >> 2, K-block tid & 3) and (row 64 + (tid >> 2), same K-block) of
+// the 128 x 128 tile: the block's amax, scale and 32 codes need no cross-lane exchange, and its 64
+// input bytes and 32 output bytes move with 256-bit accesses when the tensor is 32-byte aligned.
 
-constexpr int kSwzMaxGroups = 128;   // groups per launch; more groups are split over launches
-
-struct SwizzleArgs {
-    const uint8_t* s;         // raw scales [rows, kblocks]
-    uint8_t* out;             // swizzled output (this launch's groups start at out)
-    int64_t kblocks, ctiles;  // ctiles = ceil(kblocks / 4)
-    int ngroups;
-    int64_t src_row[kSwzMaxGroups];     // first raw row of each group
-    int64_t rows[kSwzMaxGroups];        // rows in each group
-    int64_t block_start[kSwzMaxGroups + 1];   // first output 512-byte block of each group
-};
-
-// One warp per 512-byte output block; lane l assembles 16 bytes: rows l, l+32, l+64, l+96 of the
-// block's 128-row tile, 4 K-blocks each.
-__global__ void __launch_bounds__(256) swizzle_kernel(const __grid_constant__ SwizzleArgs a) {
-    const int lane = threadIdx.x & 31;
-    const int64_t nblocks = a.block_start[a.ngroups];
-    for (int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; blk < nblocks;
-         blk += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
-        int g = 0;
-        while (g + 1 < a.ngroups && a.block_start[g + 1] <= blk) ++g;
-        const int64_t local = blk - a.block_start[g];
-        const int64_t rt = local / a.ctiles, ct = local % a.ctiles;
-        uint32_t w[4];
+__device__ __forceinline__ void load_block(const QTensor& T, int64_t row, int64_t col, bool ok, Block32& b) {
+    if (!ok) {
+        b.v[0] = b.v[1] = b.v[2] = b.v[3] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const uint16_t* p = T.x + row * T.ldx + col;
+    if (T.vec32) {
+        ld_stream_v8(p, b.v[0], b.v[1]);
+        ld_stream_v8(p + 16, b.v[2], b.v[3]);
+    } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t r = rt * 128 + lane + 32 * j;
-            uint32_t word = 0;
-            if (r < a.rows[g]) {
-                const uint8_t* src = a.s + (a.src_row[g] + r) * a.kblocks + ct * 4;
-                const int64_t nb = (a.kblocks - ct * 4 < 4 ? a.kblocks - ct * 4 : 4);
-                for (int b = 0; b < nb; ++b) word |= static_cast<uint32_t>(src[b]) << (8 * b);
+        for (int j = 0; j < 4; ++j) b.v[j] = ld_cached_v4(p + 8 * j);
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void load_row_tile(const QuantArgs<NT>& a, const TileRef& r, Block32 (&b)[2], int tid) {
+    const QTensor& T = a.t[r.i];
+    const int64_t col = r.k0 + (tid & 3) * 32;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int64_t row = r.m0 + h * 64 + (tid >> 2);
+        load_block(T, row, col, r.full || (row < T.M && col < T.K), b[h]);
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __grid_constant__ QuantArgs<NT> a) {
+    __shared__ __align__(16) uint8_t atom[512];
+    const int tid = threadIdx.x;
+
+    const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
+    const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
+    const int64_t t_end = min(a.total_tiles, t_begin + per);
+    Block32 cur[2], nxt[2];
+    TileRef rc, rn;
+    if (t_begin < t_end) {
+        rc = decode_qtile(a, t_begin);
+        load_row_tile(a, rc, cur, tid);
+    }
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        if (t + 1 < t_end) {
+            rn = rc;
+            if (++rn.kt == a.t[rn.i].tiles_k) {
+                rn.kt = 0;
+                if (++rn.mt == a.t[rn.i].tiles_m) {
+                    rn.mt = 0;
+                    ++rn.i;
+                }
             }
-            w[j] = word;
+            const QTensor& Tn = a.t[rn.i];
+            rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
+            rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
+            rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
+            load_row_tile(a, rn, nxt, tid);
         }
-        reinterpret_cast<uint4*>(a.out + blk * 512)[lane] = make_uint4(w[0], w[1], w[2], w[3]);
+        const QTensor& T = a.t[rc.i];
+        const int kb = tid & 3;
+        const int64_t col = rc.k0 + kb * 32;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = h * 64 + (tid >> 2);           // row inside the tile
+            const int64_t row = rc.m0 + r;
+            const bool valid = rc.full || (row < T.M && col < T.K);
+            const Block32& b = cur[h];
+            uint32_t m = bf16x2_absmax(bf16x2_absmax(b.v[0].x, b.v[0].y), bf16x2_absmax(b.v[0].z, b.v[0].w));
+#pragma unroll
+            for (int j = 1; j < 4; ++j)
+                m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(b.v[j].x, b.v[j].y), bf16x2_absmax(b.v[j].z, b.v[j].w)));
+            m &= 0x7FFF7FFFu;
+            const uint32_t s = scale_byte_from_amax(max(m & 0xFFFFu, m >> 16));
+            uint4 o0, o1;
+            uint2 e;
+            e = encode_chunk(b.v[0], s);
+            o0.x = e.x; o0.y = e.y;
+            e = encode_chunk(b.v[1], s);
+            o0.z = e.x; o0.w = e.y;
+            e = encode_chunk(b.v[2], s);
+            o1.x = e.x; o1.y = e.y;
+            e = encode_chunk(b.v[3], s);
+            o1.z = e.x; o1.w = e.y;
+            if (valid) {
+                uint8_t* q = T.q_row + row * T.K + col;
+                if (T.vec32) {
+                    st_v8(q, o0, o1);
+                } else {
+                    reinterpret_cast<uint4*>(q)[0] = o0;
+                    reinterpret_cast<uint4*>(q)[1] = o1;
+                }
+            }
+            atom[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
+        }
+        __syncthreads();
+        if (a.swz) {
+            if (tid < 32)
+                reinterpret_cast<uint4*>(T.s_row + (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512)[tid] =
+                    reinterpret_cast<const uint4*>(atom)[tid];
+        } else if (tid < kQTile) {
+            const int64_t kblocks = T.K / 32;
+            const int64_t m = rc.m0 + tid;
+            const int64_t nb = (kblocks - rc.kt * 4 < 4 ? kblocks - rc.kt * 4 : 4);
+            if (m < T.M)
+                for (int q = 0; q < nb; ++q)
+                    T.s_row[m * kblocks + rc.kt * 4 + q] = atom[(tid & 31) * 16 + (tid >> 5) * 4 + q];
+        }
+        __syncthreads();
+        cur[0] = nxt[0];
+        cur[1] = nxt[1];
+        rc = rn;
     }
 }
 

@@ -23,6 +23,18 @@ _STATUS = {0: "MX_OK", -1: "MX_ERR_ARG", -2: "MX_ERR_SHAPE", -3: "MX_ERR_ALIGN",
 _lib = None
 
 
+class QuantTensor(ctypes.Structure):
+    """mx_quant_tensor."""
+    _fields_ = [("x", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("ld_x", ctypes.c_int64),
+                ("q_row", ctypes.c_void_p), ("s_row", ctypes.c_void_p), ("q_col", ctypes.c_void_p),
+                ("s_col", ctypes.c_void_p)]
+
+
+class ComparePair(ctypes.Structure):
+    """mx_compare_pair."""
+    _fields_ = [("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("nbytes", ctypes.c_int64)]
+
+
 class MxError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {_STATUS.get(status, status)}")
@@ -50,6 +62,10 @@ def lib() -> ctypes.CDLL:
     L.mx_grouped_gemm.restype = I32
     L.mx_grid_equal.argtypes = [P, P, I64, P, P, P]
     L.mx_grid_equal.restype = I32
+    L.mx_quantize_multi.argtypes = [P, I64, I32, P]
+    L.mx_quantize_multi.restype = I32
+    L.mx_grid_equal_multi.argtypes = [P, I64, P, P, P]
+    L.mx_grid_equal_multi.restype = I32
     L.mx_status_string.argtypes = [I32]
     L.mx_status_string.restype = ctypes.c_char_p
     L.mx_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -104,6 +120,62 @@ def quantize(x: torch.Tensor, rowwise: bool = True, colwise: bool = False, swizz
                            ctypes.c_void_p(_stream(dev)))
     _check(st, "mx_quantize")
     return q_row, s_row, q_col, s_col
+
+
+def quant_tensor_array(xs, outs):
+    """ctypes array of mx_quant_tensor for tensors xs and their (q_row, s_row, q_col, s_col) outputs."""
+    arr = (QuantTensor * len(xs))()
+    for i, (x, (q_row, s_row, q_col, s_col)) in enumerate(zip(xs, outs)):
+        assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+        arr[i] = QuantTensor(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0),
+                             *(t.data_ptr() if t is not None else None for t in (q_row, s_row, q_col, s_col)))
+    return arr
+
+
+def quantize_multi(xs, rowwise: bool = True, colwise: bool = False, swizzle: bool = True, outs=None):
+    """mx_quantize_multi over a list of 2-D BF16 CUDA tensors (same flags); returns one
+    (q_row, s_row, q_col, s_col) tuple per tensor."""
+    if outs is None:
+        outs = []
+        for x in xs:
+            M, K = x.shape
+            u8 = dict(dtype=torch.uint8, device=x.device)
+            outs.append((
+                torch.empty((M, K), **u8) if rowwise else None,
+                (torch.empty(swizzled_scale_bytes(M, K // 32), **u8) if swizzle else torch.empty((M, K // 32), **u8))
+                if rowwise else None,
+                torch.empty((K, M), **u8) if colwise else None,
+                (torch.empty(swizzled_scale_bytes(K, M // 32), **u8) if swizzle else torch.empty((K, M // 32), **u8))
+                if colwise else None))
+    flags = (MX_ROWWISE if rowwise else 0) | (MX_COLWISE if colwise else 0) | (MX_SWIZZLE if swizzle else 0)
+    arr = quant_tensor_array(xs, outs)
+    dev = xs[0].device if xs else torch.device("cuda")
+    st = lib().mx_quantize_multi(ctypes.cast(arr, ctypes.c_void_p), len(xs), flags, ctypes.c_void_p(_stream(dev)))
+    _check(st, "mx_quantize_multi")
+    return outs
+
+
+def compare_pair_array(pairs):
+    arr = (ComparePair * len(pairs))()
+    for i, (a, b) in enumerate(pairs):
+        n = a.numel() * a.element_size()
+        assert a.is_contiguous() and b.is_contiguous() and b.numel() * b.element_size() == n
+        arr[i] = ComparePair(a.data_ptr(), b.data_ptr(), n)
+    return arr
+
+
+def grid_equal_multi(pairs, out=None):
+    """mx_grid_equal_multi over a list of (a, b) CUDA tensor pairs. Returns (mismatches, first_index):
+    int64 device tensors of len(pairs) entries (no host synchronisation)."""
+    n = len(pairs)
+    dev = pairs[0][0].device if pairs else torch.device("cuda")
+    if out is None:
+        out = torch.empty((2, max(n, 1)), dtype=torch.int64, device=dev)
+    arr = compare_pair_array(pairs)
+    st = lib().mx_grid_equal_multi(ctypes.cast(arr, ctypes.c_void_p), n, _p(out[0]), _p(out[1]),
+                                   ctypes.c_void_p(_stream(dev)))
+    _check(st, "mx_grid_equal_multi")
+    return out[0, :n], out[1, :n]
 
 
 def swizzle_scales(s: torch.Tensor, group_rows=None, out=None):

@@ -104,6 +104,23 @@ def test_swizzle_and_grid_equal_argument_errors(L):
     assert L.mx_device_error(None) == -1
 
 
+def test_multi_calls_validate_every_entry(L):
+    from mxfp8_block_scaled_07_b200 import mx
+
+    assert L.mx_quantize_multi(None, 3, 1, None) == -1
+    assert L.mx_quantize_multi(None, 0, 1, None) == 0
+    arr = (mx.QuantTensor * 2)(mx.QuantTensor(0x10000, 64, 64, 64, 0x10000, 0x10000, None, None),
+                               mx.QuantTensor(0x10000, 64, 48, 64, 0x10000, 0x10000, None, None))
+    assert L.mx_quantize_multi(ctypes.cast(arr, ctypes.c_void_p), 2, 1, None) == -2      # 2nd: K % 32
+    arr[1] = mx.QuantTensor(0x10008, 64, 64, 64, 0x10000, 0x10000, None, None)
+    assert L.mx_quantize_multi(ctypes.cast(arr, ctypes.c_void_p), 2, 1, None) == -3      # 2nd: misaligned
+    assert L.mx_quantize_multi(ctypes.cast(arr, ctypes.c_void_p), 2, 0, None) == -1      # no direction
+    pairs = (mx.ComparePair * 2)(mx.ComparePair(0x10000, 0x10000, 16), mx.ComparePair(None, 0x10000, 4))
+    assert L.mx_grid_equal_multi(ctypes.cast(pairs, ctypes.c_void_p), 2, FAKE, FAKE, None) == -1
+    assert L.mx_grid_equal_multi(ctypes.cast(pairs, ctypes.c_void_p), 1, None, FAKE, None) == -1
+    assert L.mx_grid_equal_multi(None, 0, None, None, None) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from mxfp8_block_scaled_07_b200 import mx
 

@@ -39,6 +39,35 @@ def test_random_buffers_match_oracle(n, offset):
         assert gpu_compare(a, b, offset) == oracle.grid_equal(a, b)
 
 
+def test_grid_equal_multi_matches_oracle():
+    # 700 pairs (more than one launch holds): mixed sizes, zero-length, unaligned views, faults.
+    g = np.random.default_rng(11)
+    host, pairs = [], []
+    pool_a = torch.zeros(48 << 20, dtype=torch.uint8, device="cuda")
+    pool_b = torch.zeros(48 << 20, dtype=torch.uint8, device="cuda")
+    off = 0
+    for i in range(700):
+        n = int(g.choice([0, 1, 15, 16, 100, 4096, 32768, 40000, 70001]))
+        a = synth.random_bytes(n, seed=i).numpy()
+        b = a.copy()
+        if n and g.random() < 0.5:
+            idx = g.choice(n, min(n, int(g.integers(1, 4))), replace=False)
+            b[idx] ^= np.uint8(0x81)
+        shift = int(g.integers(0, 3))         # some views start off 16-byte alignment
+        if off + shift + n > pool_a.numel():
+            break
+        pool_a[off + shift: off + shift + n] = torch.from_numpy(a)
+        pool_b[off + shift: off + shift + n] = torch.from_numpy(b)
+        pairs.append((pool_a[off + shift: off + shift + n], pool_b[off + shift: off + shift + n]))
+        host.append((a, b))
+        off += shift + n + 16 - (shift + n) % 16
+    cnt, first = mx.grid_equal_multi(pairs)
+    cnt, first = to_np(cnt), to_np(first)
+    for i, (a, b) in enumerate(host):
+        assert (int(cnt[i]), int(first[i])) == oracle.grid_equal(a, b), i
+    assert len(host) > 512
+
+
 def test_large_buffer_single_fault_at_the_end():
     # "corruption confined to ... a late layer": one byte in the last 16 bytes of 1 GiB.
     n = 1 << 30

@@ -119,6 +119,45 @@ def test_update_step_columnwise_full_size_sampled():
     assert np.array_equal(to_np(sr)[pos[rows]], so)
 
 
+@pytest.mark.parametrize("rowwise,colwise", [(True, False), (True, True), (False, True)])
+@pytest.mark.parametrize("swizzle", [True, False])
+def test_quantize_multi_matches_oracle(rowwise, colwise, swizzle):
+    # Several tensors of mixed shapes (ragged, tiny, empty, strided) in one launch.
+    shapes = [(256, 512), (32, 96), (160, 288), (0, 64), (384, 1056), (96, 32), (1024, 128)]
+    xs = []
+    for i, (M, K) in enumerate(shapes):
+        x = synth.special_bf16((M, K), seed=i) if i == 2 else synth.normal_bf16((M, K), std=2.0 ** i, seed=i,
+                                                                                 outlier_frac=0.01, outlier_scale=60.0)
+        xs.append(x)
+    dev = [x.cuda() for x in xs]
+    big = torch.zeros((384, 1096), dtype=torch.bfloat16, device="cuda")      # strided view (ld % 8 == 0)
+    big[:, :1056] = dev[4]
+    dev[4] = big[:, :1056]
+    outs = mx.quantize_multi(dev, rowwise, colwise, swizzle)
+    torch.cuda.synchronize()
+    for x, (q_row, s_row, q_col, s_col) in zip(xs, outs):
+        if x.shape[0] == 0:
+            continue
+        if rowwise:
+            q, s = oracle.quantize_rowwise(x)
+            assert np.array_equal(to_np(q_row), q)
+            assert np.array_equal(to_np(s_row), oracle.swizzle(s) if swizzle else s)
+        if colwise:
+            qT, sT = oracle.quantize_colwise(x)
+            assert np.array_equal(to_np(q_col), qT)
+            assert np.array_equal(to_np(s_col), oracle.swizzle(sT) if swizzle else sT)
+
+
+def test_quantize_multi_more_tensors_than_one_launch_holds():
+    # 400 small tensors: split over several launches inside one call.
+    xs = [synth.normal_bf16((32 * (1 + i % 5), 64 * (1 + i % 3)), seed=100 + i) for i in range(400)]
+    outs = mx.quantize_multi([x.cuda() for x in xs], True, False, True)
+    torch.cuda.synchronize()
+    for x, (q_row, s_row, _, _) in zip(xs, outs):
+        q, s = oracle.quantize_rowwise(x)
+        assert np.array_equal(to_np(q_row), q) and np.array_equal(to_np(s_row), oracle.swizzle(s))
+
+
 def test_empty_is_noop():
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q, s, _, _ = mx.quantize(x, True, False, swizzle=False)
