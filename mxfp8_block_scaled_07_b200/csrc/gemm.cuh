@@ -40,7 +40,9 @@ constexpr int kSmemA = 0;
 constexpr int kSmemB = kSmemA + kStages * kABytes;
 constexpr int kSmemSfa = kSmemB + kStages * kBBytes;
 constexpr int kSmemSfb = kSmemSfa + kStages * kSfaBytes;
-constexpr int kSmemBar = kSmemSfb + kStages * kSfbBytes;
+constexpr int kStageBytes = 32 * 128;  // epilogue staging per warp: 32 rows x 128 bytes (TMA-store box)
+constexpr int kSmemStage = kSmemSfb + kStages * kSfbBytes;            // 1024-aligned
+constexpr int kSmemBar = kSmemStage + 4 * kStageBytes;
 constexpr int kSmemMisc = kSmemBar + (2 * kStages + 3) * 8;
 constexpr int kSmemGroups = (kSmemMisc + 16 + 15) / 16 * 16;
 constexpr int kGemmSmemDense = kSmemGroups + 1024;                                  // + alignment slack
@@ -57,6 +59,7 @@ struct GemmArgs {
     int tiles_m, tiles_n;
     int out_bf16;
     int vec_store;      // output rows 16-byte aligned: full 32-column chunks use 16-byte stores
+    int tma_store;      // output written by TMA from swizzled shared-memory staging (tmap_c valid)
     int G;
     int n_rowtiles;     // ceil(N / 128): scale row-tiles of one B operand
     const int32_t* row_offsets;
@@ -105,7 +108,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int3
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                   const GemmArgs a) {
+                   const __grid_constant__ CUtensorMap tmap_c, const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSmemBar);
@@ -249,58 +252,97 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_drain(drain, 0, a.timeout_ns);
     } else {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;                 // TMEM lane quarter this warp may read
+        // Warp w reads TMEM lanes 32 * (w % 4) .. +31 (rows of the tile). The accumulator is released
+        // as soon as its last columns are in registers; rows leave through a per-warp swizzled
+        // staging buffer and a TMA store (32 rows x 128 bytes per store), or, for rows that a TMA
+        // box must not cover (a grouped tile's rows past its group) or unaligned outputs, through
+        // direct masked stores.
+        const int q = warp & 3;
         const int row_local = q * 32 + lane;
+        uint8_t* stage = smem + kSmemStage + (warp - 2) * kStageBytes;
+        const uint32_t stage_row = smem_u32(stage) + lane * 128;
+        const uint32_t swz = static_cast<uint32_t>(lane & 7);
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
             const Tile T = decode_tile<GROUPED>(t, a, off, pm);
             if (!mbar_wait(tmem_full, acc_phase, abort, a.err, a.timeout_ns)) break;
             tc_fence_after();
+            const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
+            const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
             const bool row_ok = row_local < T.rows_valid;
             const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
+            const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+            const int cols = a.out_bf16 ? 64 : 32;           // columns per 128-byte staged row
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tc_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c * 32, r);
-                tc_wait_ld();
-                const int col0 = T.n0 + c * 32;
-                if (!row_ok || col0 >= a.N) continue;
-                const int ncols = min(32, a.N - col0);
+            for (int ch = 0; ch < kBN / cols; ++ch) {
+                uint32_t p[32];                              // one 128-byte row of the chunk
                 if (a.out_bf16) {
-                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
-                    if (ncols == 32 && a.vec_store) {
-                        uint32_t p[16];
+                    uint32_t r0[32], r1[32];
+                    tc_ld_32x32b_x32(tq + ch * 64, r0);
+                    tc_ld_32x32b_x32(tq + ch * 64 + 32, r1);
+                    tc_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __nv_bfloat162 h =
-                                __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                            p[i] = *reinterpret_cast<const uint32_t*>(&h);
-                        }
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < ncols) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+                        p[i] = *reinterpret_cast<const uint32_t*>(&h0);
+                        p[16 + i] = *reinterpret_cast<const uint32_t*>(&h1);
                     }
                 } else {
-                    float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
-                    if (ncols == 32 && a.vec_store) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
+                    tc_ld_32x32b_x32(tq + ch * 32, p);
+                    tc_wait_ld();
+                }
+                if (ch == kBN / cols - 1) {
+                    tc_fence_before();
+                    mbar_arrive(tmem_empty);                 // accumulator free for the next tile
+                }
+                const int col0 = T.n0 + ch * cols;
+                if (col0 >= a.N) continue;
+                if (use_tma) {
+                    if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
+                    __syncwarp();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) d4[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    for (int j = 0; j < 8; ++j)
+                        st_shared_v4(stage_row + ((static_cast<uint32_t>(j) ^ swz) << 4), p[4 * j], p[4 * j + 1],
+                                     p[4 * j + 2], p[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_c, stage, col0, T.a_row0 + q * 32);
+                        bulk_commit_group();
+                    }
+                } else if (row_ok) {
+                    const int ncols = min(cols, a.N - col0);
+                    if (a.out_bf16) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
+                        if (ncols == cols && a.vec_store) {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 64; ++i)
+                                if (i < ncols)
+                                    dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
+                        }
                     } else {
+                        float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
+                        if (ncols == cols && a.vec_store) {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < ncols) dst[i] = __uint_as_float(r[i]);
+                            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < ncols) dst[i] = __uint_as_float(p[i]);
+                        }
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(tmem_empty);
             acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_group<0>();                 // every TMA store of this warp complete
+        __syncwarp();
     }
 
     tc_fence_before();

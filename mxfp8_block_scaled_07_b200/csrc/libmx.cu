@@ -112,8 +112,8 @@ mx_status check_device(const DeviceInfo** out) {
 
 mx_status launched() { return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 
-bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t rows, uint32_t box_cols,
-               uint32_t box_rows) {
+// cuTensorMapEncodeTiled from the driver, looked up once (no link-time dependency on libcuda).
+EncodeTiledFn encode_fn() {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -121,7 +121,14 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t
             q == cudaDriverEntryPointSuccess)
             g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     });
-    if (!g_encode) return false;
+    return g_encode;
+}
+
+// Tensor map of a K-major E4M3 operand [rows, cols_bytes]: boxes of box_rows x box_cols bytes with
+// the 128-byte swizzle the UMMA descriptors expect.
+bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t rows, uint32_t box_cols,
+               uint32_t box_rows) {
+    if (!encode_fn()) return false;
     const cuuint64_t dims[2] = {cols_bytes, rows};
     const cuuint64_t strides[1] = {cols_bytes};
     const cuuint32_t box[2] = {box_cols, box_rows};
@@ -132,6 +139,24 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Tensor map for the GEMM output C[rows, N] (row stride ld_c elements) written by the epilogue's
+// TMA stores: 32-row boxes of 128 bytes (64 BF16 or 32 fp32 columns), 128-byte swizzle. Returns
+// false (and the epilogue uses direct stores) when C's base or row stride is not 16-byte aligned.
+bool make_tmap_out(CUtensorMap* map, const void* c, int64_t rows, int64_t N, int64_t ld_c, mx_out_dtype dt) {
+    std::memset(map, 0, sizeof *map);
+    const int64_t esz = dt == MX_OUT_BF16 ? 2 : 4;
+    if (!aligned16(c) || (ld_c * esz) % 16 != 0) return false;
+    if (!encode_fn()) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_c * esz)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, dt == MX_OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                    const_cast<void*>(c), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // Checks shared by both GEMMs. Sets *empty when there is nothing to compute (then pointers may be
 // null). The output may have any element alignment; 16-byte aligned rows take vector stores.
@@ -433,6 +458,8 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     a.tiles_n = static_cast<int>(ceil_div(N, kBN));
     a.out_bf16 = out_dtype == MX_OUT_BF16;
     a.vec_store = vector_store_ok(c, ld_c, out_dtype);
+    CUtensorMap tc;
+    a.tma_store = make_tmap_out(&tc, c, M, N, ld_c, out_dtype);
     a.G = 1;
     a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
     a.row_offsets = nullptr;
@@ -440,7 +467,7 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     a.timeout_ns = g_timeout_ns.load();
     const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, d->sms));
-    mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, a);
+    mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, tc, a);
     return launched();
 }
 
@@ -473,6 +500,8 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     a.tiles_n = static_cast<int>(ceil_div(N, kBN));
     a.out_bf16 = out_dtype == MX_OUT_BF16;
     a.vec_store = vector_store_ok(c, ld_c, out_dtype);
+    CUtensorMap tc;
+    a.tma_store = make_tmap_out(&tc, c, total_rows, N, ld_c, out_dtype);
     a.G = static_cast<int>(G);
     a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
     a.row_offsets = row_offsets_dev;
@@ -481,7 +510,7 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     // Upper bound on tiles: every group adds at most one partial 128-row tile.
     const int64_t max_tiles = (ceil_div(total_rows, kBM) + G) * a.tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, d->sms));
-    mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, a);
+    mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, tc, a);
     return launched();
 }
 
