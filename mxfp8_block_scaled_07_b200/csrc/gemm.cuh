@@ -272,32 +272,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row_local < T.rows_valid;
             const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
             const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-            const int cols = a.out_bf16 ? 64 : 32;           // columns per 128-byte staged row
-#pragma unroll 1
-            for (int ch = 0; ch < kBN / cols; ++ch) {
-                uint32_t p[32];                              // one 128-byte row of the chunk
-                if (a.out_bf16) {
-                    uint32_t r0[32], r1[32];
-                    tc_ld_32x32b_x32(tq + ch * 64, r0);
-                    tc_ld_32x32b_x32(tq + ch * 64 + 32, r1);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
-                        p[i] = *reinterpret_cast<const uint32_t*>(&h0);
-                        p[16 + i] = *reinterpret_cast<const uint32_t*>(&h1);
-                    }
-                } else {
-                    tc_ld_32x32b_x32(tq + ch * 32, p);
-                    tc_wait_ld();
-                }
-                if (ch == kBN / cols - 1) {
-                    tc_fence_before();
-                    mbar_arrive(tmem_empty);                 // accumulator free for the next tile
-                }
-                const int col0 = T.n0 + ch * cols;
-                if (col0 >= a.N) continue;
+            // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of this
+            // warp's 32 rows.
+            auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
+                if (col0 >= a.N) return;
                 if (use_tma) {
                     if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
                     __syncwarp();
@@ -313,30 +291,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 } else if (row_ok) {
                     const int ncols = min(cols, a.N - col0);
-                    if (a.out_bf16) {
+                    if (ncols == cols && a.vec_store) {
+                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.c) +
+                                                             (crow * a.ldc + col0) * (a.out_bf16 ? 2 : 4));
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+                    } else if (a.out_bf16) {
                         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
-                        if (ncols == cols && a.vec_store) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 64; ++i)
-                                if (i < ncols)
-                                    dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
-                        }
+                        for (int i = 0; i < 64; ++i)
+                            if (i < ncols) dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
                     } else {
                         float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
-                        if (ncols == cols && a.vec_store) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i < ncols) dst[i] = __uint_as_float(p[i]);
-                        }
+                        for (int i = 0; i < 32; ++i)
+                            if (i < ncols) dst[i] = __uint_as_float(p[i]);
                     }
+                }
+            };
+            if (a.out_bf16) {
+                // All 256 columns into registers (packed BF16), then release the accumulator.
+                uint32_t pk[4][32];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t r[32];
+                    tc_ld_32x32b_x32(tq + ch * 32, r);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        pk[ch >> 1][(ch & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tmem_empty);                     // accumulator free for the next tile
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) emit(pk[ch], T.n0 + ch * 64, 64);
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < kBN / 32; ++ch) {
+                    uint32_t p[32];
+                    tc_ld_32x32b_x32(tq + ch * 32, p);
+                    tc_wait_ld();
+                    if (ch == kBN / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(tmem_empty);
+                    }
+                    emit(p, T.n0 + ch * 32, 32);
                 }
             }
             acc_phase ^= 1u;
