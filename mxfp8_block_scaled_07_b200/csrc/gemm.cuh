@@ -34,7 +34,11 @@ constexpr int kSfbBytes = 1024;
 constexpr int kGemmThreads = 192;
 constexpr int kMaxGroups = 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = kBN;  // fp32 accumulator: 256 TMEM columns x 128 lanes
+// TMEM columns (x 128 lanes, 32-bit): accumulator 0 = [0, 256), accumulator 1 = [240, 496) (the two
+// share [240, 256)), scale slot = [496, 508): A scales 4 columns, B scales 8 columns.
+constexpr uint32_t kAcc1Col = 240;
+constexpr uint32_t kOvlCol = 240;
+constexpr uint32_t kSfCol = 496;
 
 constexpr int kSmemA = 0;
 constexpr int kSmemB = kSmemA + kStages * kABytes;
@@ -114,8 +118,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSmemBar);
     uint64_t* empty = full + kStages;
     uint64_t* tmem_full = empty + kStages;
-    uint64_t* tmem_empty = tmem_full + 1;
-    uint64_t* drain = tmem_empty + 1;
+    uint64_t* ovl_free = tmem_full + 1;     // epilogue has drained the shared accumulator columns
+    uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + kSmemMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
     int* total_tiles = reinterpret_cast<int*>(smem + kSmemMisc + 8);
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 4 * 32);
+        mbar_init(ovl_free, 4 * 32);
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -210,19 +214,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        // Tile j accumulates into TMEM columns [acc_j, acc_j + 256): acc_j = 0 for even j, 240 for odd
+        // j. The two accumulators share columns 240-255, which the epilogue reads first; tile j starts
+        // as soon as those of tile j-1 are drained (by then the epilogue has finished tile j-2). The
+        // scale blocks go to one TMEM slot (columns 496-507): tcgen05 operations issued by one thread
+        // execute in order, so a copy never overtakes the MMAs that read the previous contents.
         int stage = 0;
-        uint32_t phase = 0, acc_phase = 0;
+        uint32_t phase = 0, ovl_phase = 0;
         bool ok = true;
-        const uint32_t sfa_base = tmem_base + kAccCols;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            if (!mbar_wait(tmem_empty, acc_phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
+        const uint32_t sfa_t = tmem_base + kSfCol;
+        const uint32_t sfb_t = sfa_t + 4;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+            if (j > 0) {
+                if (!mbar_wait(ovl_free, ovl_phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
+                ovl_phase ^= 1u;
+            }
             tc_fence_after();
+            const uint32_t acc = tmem_base + ((j & 1) ? kAcc1Col : 0u);
             for (int kb = 0; kb < a.nkb; ++kb) {
                 if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t sfa_t = sfa_base + stage * 16;
-                    const uint32_t sfb_t = sfa_t + 4;
                     tc_cp_32x128b_warpx4(sfa_t, sdesc_scale_block(smem_u32(smem + kSmemSfa + stage * kSfaBytes)));
                     tc_cp_32x128b_warpx4(sfb_t, sdesc_scale_block(smem_u32(smem + kSmemSfb + stage * kSfbBytes)));
                     tc_cp_32x128b_warpx4(sfb_t + 4,
@@ -232,7 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         // K-step k: +32 bytes inside the 128-byte swizzled rows; scale byte k.
-                        tc_mma_mxf8(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(kBM, kBN, k),
+                        tc_mma_mxf8(acc, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(kBM, kBN, k),
                                     sfa_t | (static_cast<uint32_t>(k) << 30), sfb_t | (static_cast<uint32_t>(k) << 30),
                                     (kb | k) != 0 ? 1u : 0u);
                     }
@@ -244,7 +257,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!ok) break;
             if (lane == 0) tc_commit(tmem_full);
             __syncwarp();
-            acc_phase ^= 1u;
         }
         // Every MMA issued by this thread has completed once `drain` fires.
         if (lane == 0) tc_commit(drain);
@@ -262,16 +274,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* stage = smem + kSmemStage + (warp - 2) * kStageBytes;
         const uint32_t stage_row = smem_u32(stage) + lane * 128;
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        uint32_t full_phase = 0;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             const Tile T = decode_tile<GROUPED>(t, a, off, pm);
-            if (!mbar_wait(tmem_full, acc_phase, abort, a.err, a.timeout_ns)) break;
+            if (!mbar_wait(tmem_full, full_phase, abort, a.err, a.timeout_ns)) break;
+            full_phase ^= 1u;
             tc_fence_after();
             const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
             const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
             const bool row_ok = row_local < T.rows_valid;
             const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
-            const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+            const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+            const bool acc1 = (j & 1) != 0;
+            const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
+            // The shared columns first (tile columns 240..255 of accumulator 0, 0..15 of accumulator
+            // 1); once every epilogue thread has them, the next tile's MMAs may start.
+            uint32_t ov[16];
+            tc_ld_32x32b_x16(lanes + kOvlCol, ov);
+            tc_wait_ld();
+            tc_fence_before();
+            mbar_arrive(ovl_free);
             // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of this
             // warp's 32 rows.
             auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
@@ -280,9 +303,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
                     __syncwarp();
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        st_shared_v4(stage_row + ((static_cast<uint32_t>(j) ^ swz) << 4), p[4 * j], p[4 * j + 1],
-                                     p[4 * j + 2], p[4 * j + 3]);
+                    for (int i = 0; i < 8; ++i)
+                        st_shared_v4(stage_row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1],
+                                     p[4 * i + 2], p[4 * i + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -309,38 +332,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             };
-            if (a.out_bf16) {
-                // All 256 columns into registers (packed BF16), then release the accumulator.
-                uint32_t pk[4][32];
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t r[32];
-                    tc_ld_32x32b_x32(tq + ch * 32, r);
+            // Columns [c * 16, c * 16 + 32) for even c: from the shared columns already in `ov` where
+            // they fall there, else from TMEM.
+            auto fetch32 = [&](int c, uint32_t(&p)[32]) {
+                const bool lo_shared = acc1 && c == 0;          // tile columns 0..15 of accumulator 1
+                const bool hi_shared = !acc1 && c == 14;        // tile columns 240..255 of accumulator 0
+                if (lo_shared || hi_shared) {
+                    uint32_t r[16];
+                    tc_ld_32x32b_x16(tq + (lo_shared ? 16u : 224u), r);
                     tc_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
+                        p[i] = lo_shared ? ov[i] : r[i];
+                        p[16 + i] = lo_shared ? r[i] : ov[i];
+                    }
+                } else {
+                    tc_ld_32x32b_x32(tq + c * 16, p);
+                    tc_wait_ld();
+                }
+            };
+            if (a.out_bf16) {
+                uint32_t pk[4][32];                          // the row's 256 columns, packed BF16
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
+                    uint32_t r[32];
+                    fetch32(c, r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
                         __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                        pk[ch >> 1][(ch & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+                        pk[c >> 2][((c >> 1) & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(tmem_empty);                     // accumulator free for the next tile
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) emit(pk[ch], T.n0 + ch * 64, 64);
             } else {
-#pragma unroll 1
-                for (int ch = 0; ch < kBN / 32; ++ch) {
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
                     uint32_t p[32];
-                    tc_ld_32x32b_x32(tq + ch * 32, p);
-                    tc_wait_ld();
-                    if (ch == kBN / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(tmem_empty);
-                    }
-                    emit(p, T.n0 + ch * 32, 32);
+                    fetch32(c, p);
+                    emit(p, T.n0 + c * 16, 32);
                 }
             }
-            acc_phase ^= 1u;
         }
         if (lane == 0) bulk_wait_group<0>();                 // every TMA store of this warp complete
         __syncwarp();
