@@ -531,6 +531,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", choices=CASES, help="run one kernel config only (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1],
+                    help="GEMM kernel for --case runs: 0 CTA pair (default), 1 single CTA")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -540,6 +542,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.case:
+        from mxfp8_block_scaled_07_b200 import build as mxbuild
+        from mxfp8_block_scaled_07_b200 import mx
+
+        mxbuild.build()
+        mx.set_gemm_variant(args.gemm_variant)
         return run_case(args.case, args.reps)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

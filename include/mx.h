@@ -154,6 +154,14 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
                           mx_out_dtype out_dtype, mx_stream stream);
 
 /*
+ * Selects the kernel behind later mx_gemm / mx_grouped_gemm calls (process-wide): 0 (default) the
+ * CTA-pair kernel (256 x 256 tiles computed by two SMs with tcgen05.mma.cta_group::2), 1 the
+ * single-CTA kernel (128 x 256 tiles). Both meet the accuracy bound above; results may differ in
+ * fp32 summation order only. Other values select 0.
+ */
+void mx_set_gemm_variant(int variant);
+
+/*
  * Byte comparison (abstract and Table 11: the synchronized sampler weights, scales and kernel
  * layout must equal the learner's quantization byte for byte): counts the positions i < nbytes
  * with a[i] != b[i] and finds the smallest such i. Results are written to device memory:

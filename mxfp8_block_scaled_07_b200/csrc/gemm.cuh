@@ -7,28 +7,36 @@
 // on Blackwell" (Table 6: GEMM 20.4 ms BF16 vs 13.3 ms MXFP8 per micro-batch; Table 2: dense
 // Qwen3-8B and the 128-expert Qwen3-30B-A3B MoE, whose expert GEMMs run grouped).
 //
-// Design (one CTA per SM, persistent, static tile schedule, warp-specialized):
-//   warp 0     TMA producer: A tile 128 x 128 B, B tile 256 x 128 B (128-byte swizzle), and the
-//              512-byte scale blocks (1 for A, 2 for B) by bulk copy, into a 4-stage ring;
-//   warp 1     TMEM owner and MMA issuer: per stage, tcgen05.cp of the scale blocks into TMEM,
-//              then 4 MMAs of 128 x 256 x 32 (one per 32-K block, selecting its scale byte);
-//   warps 2-5  epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator (warp w reads TMEM lanes
-//              32 * (w % 4) ..), convert, store to global.
-// Every mbarrier wait is bounded (globaltimer deadline); on expiry the kernel records an error
-// bit, stops all roles, drains its in-flight copies and MMAs, frees TMEM and returns.
+// Two kernels, both persistent with a static tile schedule and warp specialization:
+//
+//   mx_gemm_pair_kernel (default): a cluster of 2 CTAs on two SMs computes a 256 x 256 tile with
+//     tcgen05.mma.cta_group::2 (M = 256, N = 256). Each CTA loads its own 128 rows of A, half of B's
+//     256 rows and the full 256-row B scale tile; the leader CTA issues the scale copies and MMAs for
+//     both. Per SM this halves B traffic and the scale-copy work per FLOP against one CTA alone.
+//   mx_gemm_kernel: one CTA computes a 128 x 256 tile with cta_group::1 MMAs.
+//
+// Roles (192 threads): warp 0 TMA producer (A/B tiles with the 128-byte swizzle, scale blocks);
+// warp 1 TMEM owner and MMA issuer; warps 2-5 epilogue (warp w reads TMEM lanes 32 * (w % 4)).
+// TMEM: two accumulators overlapping in 16 columns ([0, 256) and [240, 496)) and one scale slot
+// ([496, 508)): the epilogue drains the shared columns first, so the next tile's MMAs start while
+// the rest of the previous tile is still being read out. tcgen05 operations issued by one thread
+// execute in order, so a scale copy never overtakes the MMAs that read the slot's previous contents.
+// The epilogue writes through per-warp swizzled staging and TMA stores.
+//
+// Every mbarrier wait is bounded (globaltimer deadline); on expiry the kernel records an error bit,
+// stops all roles, drains its in-flight copies and MMAs, frees TMEM and returns. No load uses
+// cluster multicast.
 #pragma once
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 
 namespace mx {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBM = 128;            // rows of A per CTA
+constexpr int kBN = 256;            // columns of C per tile
 constexpr int kBK = 128;            // bytes of K per stage (= one 128-byte swizzle row)
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK;  // 16 KB
-constexpr int kBBytes = kBN * kBK;  // 32 KB
 constexpr int kSfaBytes = 512;
 constexpr int kSfbBytes = 1024;
 constexpr int kGemmThreads = 192;
@@ -39,18 +47,37 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 240;
 constexpr uint32_t kOvlCol = 240;
 constexpr uint32_t kSfCol = 496;
-
-constexpr int kSmemA = 0;
-constexpr int kSmemB = kSmemA + kStages * kABytes;
-constexpr int kSmemSfa = kSmemB + kStages * kBBytes;
-constexpr int kSmemSfb = kSmemSfa + kStages * kSfaBytes;
 constexpr int kStageBytes = 32 * 128;  // epilogue staging per warp: 32 rows x 128 bytes (TMA-store box)
-constexpr int kSmemStage = kSmemSfb + kStages * kSfbBytes;            // 1024-aligned
-constexpr int kSmemBar = kSmemStage + 4 * kStageBytes;
-constexpr int kSmemMisc = kSmemBar + (2 * kStages + 3) * 8;
-constexpr int kSmemGroups = (kSmemMisc + 16 + 15) / 16 * 16;
-constexpr int kGemmSmemDense = kSmemGroups + 1024;                                  // + alignment slack
-constexpr int kGemmSmemGrouped = kSmemGroups + 2 * (kMaxGroups + 1) * 4 + 1024;
+
+// Shared-memory layout of one kernel configuration. B_ROWS: rows of B per CTA and stage.
+template <int STAGES, int B_ROWS, int GROUP_ARRAYS>
+struct GemmSmem {
+    static constexpr int kA = 0;
+    static constexpr int kB = kA + STAGES * kBM * kBK;
+    static constexpr int kSfa = kB + STAGES * B_ROWS * kBK;
+    static constexpr int kSfb = kSfa + STAGES * kSfaBytes;
+    // The staging buffers must start on a 1024-byte boundary: the 128-byte swizzle the TMA store
+    // applies is a function of the address bits 7-9.
+    static constexpr int kStage = (kSfb + STAGES * kSfbBytes + 1023) / 1024 * 1024;
+    static_assert(kA % 1024 == 0 && kB % 1024 == 0 && kStage % 1024 == 0, "swizzled buffers 1024-aligned");
+    static constexpr int kBar = kStage + 4 * kStageBytes;
+    static constexpr int kMisc = kBar + (2 * STAGES + 3) * 8;
+    static constexpr int kGroups = (kMisc + 16 + 15) / 16 * 16;
+    static constexpr int kBytes = kGroups + GROUP_ARRAYS * (kMaxGroups + 1) * 4 + 1024;   // + alignment slack
+};
+constexpr int kStages1 = 4;                 // single-CTA kernel
+constexpr int kStagesPairDense = 6;         // pair kernel
+constexpr int kStagesPairGrouped = 5;
+using Smem1Dense = GemmSmem<kStages1, kBN, 0>;
+using Smem1Grouped = GemmSmem<kStages1, kBN, 2>;
+using SmemPairDense = GemmSmem<kStagesPairDense, kBN / 2, 0>;
+using SmemPairGrouped = GemmSmem<kStagesPairGrouped, kBN / 2, 3>;
+constexpr int kGemmSmemDense = Smem1Dense::kBytes;
+constexpr int kGemmSmemGrouped = Smem1Grouped::kBytes;
+constexpr int kGemmPairSmemDense = SmemPairDense::kBytes;
+constexpr int kGemmPairSmemGrouped = SmemPairGrouped::kBytes;
+static_assert(kGemmPairSmemDense <= 232448 && kGemmPairSmemGrouped <= 232448 && kGemmSmemGrouped <= 232448,
+              "shared memory per CTA");
 
 struct GemmArgs {
     const uint8_t* sfa;
@@ -60,7 +87,9 @@ struct GemmArgs {
     int M;              // dense: rows of A; grouped: total rows
     int N, K;
     int nkb;            // ceil(K / 128)
-    int tiles_m, tiles_n;
+    int tiles_m;        // dense: row tiles (128 rows single-CTA, 256 rows pair)
+    int tiles_n;        // 256-column tiles
+    int sfa_tiles;      // 128-row tiles in A's scale layout (dense), for clamping
     int out_bf16;
     int vec_store;      // output rows 16-byte aligned: full 32-column chunks use 16-byte stores
     int tma_store;      // output written by TMA from swizzled shared-memory staging (tmap_c valid)
@@ -71,17 +100,29 @@ struct GemmArgs {
     uint64_t timeout_ns;
 };
 
+// What one CTA does for one tile.
 struct Tile {
-    int a_row0;         // first A row (TMA coordinate)
-    int rows_valid;     // rows of C this tile owns
-    int b_row0;         // first B row (TMA coordinate)
+    int a_row0;         // first A row of this CTA (TMA coordinate; also first C row)
+    int rows_valid;     // rows of C this CTA owns in the tile (0..128)
+    int b_row0;         // first B row this CTA loads (TMA coordinate)
     int n0;             // first output column
     int sfa_tile;       // 128-row tile index into A's scale layout
-    int sfb_tile;       // 128-row tile index into B's scale layout
+    int sfb_tile0;      // 128-row tile indices into B's scale layout (columns n0.., n0 + 128..)
+    int sfb_tile1;
 };
 
+// Largest g in [0, G) with pm[g] <= x (pm nondecreasing, x < pm[G]).
+__device__ __forceinline__ int find_group(const int32_t* pm, int G, int x) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pm[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 template <bool GROUPED>
-__device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int32_t* off, const int32_t* pm) {
+__device__ __forceinline__ Tile decode_tile1(int t, const GemmArgs& a, const int32_t* off, const int32_t* pm) {
     Tile T;
     if constexpr (!GROUPED) {
         const int mt = t % a.tiles_m, nt = t / a.tiles_m;
@@ -90,52 +131,220 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int3
         T.n0 = nt * kBN;
         T.b_row0 = T.n0;
         T.sfa_tile = mt;
-        T.sfb_tile = T.n0 / 128;
+        T.sfb_tile0 = T.n0 / 128;
     } else {
         const int mtg = t / a.tiles_n, nt = t % a.tiles_n;
-        int lo = 0, hi = a.G - 1;      // largest g with pm[g] <= mtg
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (pm[mid] <= mtg) lo = mid; else hi = mid - 1;
-        }
-        const int g = lo;
+        const int g = find_group(pm, a.G, mtg);
         T.a_row0 = off[g] + (mtg - pm[g]) * kBM;
         T.rows_valid = min(kBM, off[g + 1] - T.a_row0);
         T.n0 = nt * kBN;
         T.b_row0 = g * a.N + T.n0;
         T.sfa_tile = mtg;
-        T.sfb_tile = g * a.n_rowtiles + T.n0 / 128;
+        T.sfb_tile0 = g * a.n_rowtiles + T.n0 / 128;
     }
+    T.sfb_tile1 = T.sfb_tile0 + 1;
     return T;
 }
 
+// Pair tiles are 256 x 256; CTA `rank` owns rows [128 rank, 128 rank + 128) of the tile and loads B
+// rows [n0 + 128 rank, +128). Scale-tile indices past the real ones are clamped to valid memory;
+// those rows / columns are never written.
+template <bool GROUPED>
+__device__ __forceinline__ Tile decode_tile_pair(int t, int rank, const GemmArgs& a, const int32_t* off,
+                                                 const int32_t* pm128, const int32_t* pm256) {
+    Tile T;
+    int sf_last_in_b;
+    if constexpr (!GROUPED) {
+        const int mt = t % a.tiles_m, nt = t / a.tiles_m;
+        T.a_row0 = mt * 2 * kBM + rank * kBM;
+        T.rows_valid = max(0, min(kBM, a.M - T.a_row0));
+        T.n0 = nt * kBN;
+        T.b_row0 = T.n0 + rank * kBM;
+        T.sfa_tile = min(2 * mt + rank, a.sfa_tiles - 1);
+        T.sfb_tile0 = T.n0 / 128;
+        sf_last_in_b = a.n_rowtiles - 1;
+    } else {
+        const int mtg = t / a.tiles_n, nt = t % a.tiles_n;
+        const int g = find_group(pm256, a.G, mtg);
+        const int local = mtg - pm256[g];
+        T.a_row0 = off[g] + local * 2 * kBM + rank * kBM;
+        T.rows_valid = max(0, min(kBM, off[g + 1] - T.a_row0));
+        T.n0 = nt * kBN;
+        T.b_row0 = g * a.N + T.n0 + rank * kBM;
+        T.sfa_tile = min(pm128[g] + 2 * local + rank, pm128[a.G] - 1);
+        T.sfb_tile0 = g * a.n_rowtiles + T.n0 / 128;
+        sf_last_in_b = g * a.n_rowtiles + a.n_rowtiles - 1;
+    }
+    T.sfb_tile1 = min(T.sfb_tile0 + 1, sf_last_in_b);
+    return T;
+}
+
+// Reads the fp32 accumulator of one tile (this warp's 32 TMEM lanes = 32 rows) and writes C.
+// The columns shared by the two accumulators are read first; then one arrive per warp on the
+// `ovl_free` barrier (shared::cluster address) tells the MMA issuer it may start the next tile.
+// Rows leave through the warp's swizzled staging buffer and a TMA store (32 rows x 128 bytes), or,
+// where a TMA box must not go (a grouped tile's rows past its group) or the output is not aligned
+// for TMA, through direct masked stores.
+template <bool GROUPED>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorMap* tmap_c, const Tile& T,
+                                              uint32_t tmem_base, bool acc1, uint8_t* stage, uint32_t ovl_free_addr,
+                                              int q, int lane) {
+    const int row_local = q * 32 + lane;
+    const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
+    const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
+    const bool row_ok = row_local < T.rows_valid;
+    const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
+    const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
+    const uint32_t stage_row = smem_u32(stage) + lane * 128;
+    const uint32_t swz = static_cast<uint32_t>(lane & 7);
+
+    uint32_t ov[16];                     // tile columns 240..255 of accumulator 0, 0..15 of accumulator 1
+    tc_ld_32x32b_x16(lanes + kOvlCol, ov);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
+
+    // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of the 32 rows.
+    auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
+        if (col0 >= a.N) return;
+        if (use_tma) {
+            if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                st_shared_v4(stage_row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1], p[4 * i + 2],
+                             p[4 * i + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmap_c, stage, col0, T.a_row0 + q * 32);
+                bulk_commit_group();
+            }
+        } else if (row_ok) {
+            const int ncols = min(cols, a.N - col0);
+            if (ncols == cols && a.vec_store) {
+                uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.c) +
+                                                     (crow * a.ldc + col0) * (a.out_bf16 ? 2 : 4));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            } else if (a.out_bf16) {
+                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (i < ncols) dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
+            } else {
+                float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < ncols) dst[i] = __uint_as_float(p[i]);
+            }
+        }
+    };
+    // Tile columns [c * 16, c * 16 + 32) for even c: from `ov` where they are the shared columns,
+    // else from TMEM.
+    auto fetch32 = [&](int c, uint32_t(&p)[32]) {
+        const bool lo_shared = acc1 && c == 0;
+        const bool hi_shared = !acc1 && c == 14;
+        if (lo_shared || hi_shared) {
+            uint32_t r[16];
+            tc_ld_32x32b_x16(tq + (lo_shared ? 16u : 224u), r);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                p[i] = lo_shared ? ov[i] : r[i];
+                p[16 + i] = lo_shared ? r[i] : ov[i];
+            }
+        } else {
+            tc_ld_32x32b_x32(tq + c * 16, p);
+            tc_wait_ld();
+        }
+    };
+    if (a.out_bf16) {
+        uint32_t pk[4][32];                  // the row's 256 columns, packed BF16
+#pragma unroll
+        for (int c = 0; c < 16; c += 2) {
+            uint32_t r[32];
+            fetch32(c, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                pk[c >> 2][((c >> 1) & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) emit(pk[ch], T.n0 + ch * 64, 64);
+    } else {
+#pragma unroll
+        for (int c = 0; c < 16; c += 2) {
+            uint32_t p[32];
+            fetch32(c, p);
+            emit(p, T.n0 + c * 16, 32);
+        }
+    }
+}
+
+// Loads the group row offsets into shared memory, checks them and builds the prefix sums of
+// row tiles per group (tile_rows = 128: pm128; also 256: pm256 when given). Returns the tile count
+// (0 and an error bit when the offsets are invalid). Executed by the whole CTA.
+__device__ __forceinline__ int setup_groups(const GemmArgs& a, int32_t* off, int32_t* pm128, int32_t* pm256,
+                                            int tiles_n) {
+    for (int g = threadIdx.x; g <= a.G; g += blockDim.x) off[g] = a.row_offsets[g];
+    __syncthreads();
+    __shared__ int total;
+    if (threadIdx.x == 0) {
+        bool ok = off[0] == 0 && off[a.G] == a.M;
+        int acc128 = 0, acc256 = 0;
+        for (int g = 0; g < a.G; ++g) {
+            pm128[g] = acc128;
+            if (pm256) pm256[g] = acc256;
+            const int n = off[g + 1] - off[g];
+            if (n < 0) ok = false;
+            acc128 += n > 0 ? (n + 127) / 128 : 0;
+            acc256 += n > 0 ? (n + 255) / 256 : 0;
+        }
+        pm128[a.G] = acc128;
+        if (pm256) pm256[a.G] = acc256;
+        if (!ok) atomicOr(a.err, kErrBadOffsets);
+        total = ok ? (pm256 ? acc256 : acc128) * tiles_n : 0;
+    }
+    __syncthreads();
+    return total;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Single-CTA kernel: 128 x 256 tiles.
+// ---------------------------------------------------------------------------------------------
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_c, const GemmArgs a) {
+    using L = typename std::conditional<GROUPED, Smem1Grouped, Smem1Dense>::type;
+    constexpr int S = kStages1;
+    constexpr int kBBytes = kBN * kBK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSmemBar);
-    uint64_t* empty = full + kStages;
-    uint64_t* tmem_full = empty + kStages;
-    uint64_t* ovl_free = tmem_full + 1;     // epilogue has drained the shared accumulator columns
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* empty = full + S;
+    uint64_t* tmem_full = empty + S;
+    uint64_t* ovl_free = tmem_full + 1;     // the epilogue has drained the shared accumulator columns
     uint64_t* drain = ovl_free + 1;
-    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + kSmemMisc);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
-    int* total_tiles = reinterpret_cast<int*>(smem + kSmemMisc + 8);
-    int32_t* off = reinterpret_cast<int32_t*>(smem + kSmemGroups);
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    int32_t* off = reinterpret_cast<int32_t*>(smem + L::kGroups);
     int32_t* pm = off + (kMaxGroups + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(ovl_free, 4 * 32);
+        mbar_init(ovl_free, 4);
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -148,30 +357,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_alloc(tmem_base_slot, kTmemCols);
         tmem_relinquish();
     }
-    if constexpr (GROUPED) {
-        for (int g = threadIdx.x; g <= a.G; g += blockDim.x) off[g] = a.row_offsets[g];
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            bool ok = off[0] == 0 && off[a.G] == a.M;
-            int acc = 0;
-            for (int g = 0; g < a.G; ++g) {
-                pm[g] = acc;
-                const int n = off[g + 1] - off[g];
-                if (n < 0) ok = false;
-                acc += n > 0 ? (n + kBM - 1) / kBM : 0;
-            }
-            pm[a.G] = acc;
-            if (!ok) atomicOr(a.err, kErrBadOffsets);
-            *total_tiles = ok ? acc * a.tiles_n : 0;
-        }
-    } else {
-        if (threadIdx.x == 0) *total_tiles = a.tiles_m * a.tiles_n;
-    }
+    int tiles;
+    if constexpr (GROUPED)
+        tiles = setup_groups(a, off, pm, nullptr, a.tiles_n);
+    else
+        tiles = a.tiles_m * a.tiles_n;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
-    const int tiles = *total_tiles;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -180,45 +374,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int issued = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const Tile T = decode_tile<GROUPED>(t, a, off, pm);
+            const Tile T = decode_tile1<GROUPED>(t, a, off, pm);
             const bool sfb1 = T.n0 + 128 < a.N;
-            const uint32_t bytes = kABytes + kBBytes + kSfaBytes + (sfb1 ? 1024u : 512u);
+            const uint32_t bytes = kBM * kBK + kBBytes + kSfaBytes + (sfb1 ? 1024u : 512u);
             for (int kb = 0; kb < a.nkb; ++kb) {
                 if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[stage], bytes);
-                    tma_load_2d(smem + kSmemA + stage * kABytes, &tmap_a, &full[stage], kb * kBK, T.a_row0);
-                    tma_load_2d(smem + kSmemB + stage * kBBytes, &tmap_b, &full[stage], kb * kBK, T.b_row0);
-                    bulk_load(smem + kSmemSfa + stage * kSfaBytes,
-                              a.sfa + (static_cast<int64_t>(T.sfa_tile) * a.nkb + kb) * 512, 512, &full[stage]);
-                    bulk_load(smem + kSmemSfb + stage * kSfbBytes,
-                              a.sfb + (static_cast<int64_t>(T.sfb_tile) * a.nkb + kb) * 512, 512, &full[stage]);
-                    if (sfb1)
-                        bulk_load(smem + kSmemSfb + stage * kSfbBytes + 512,
-                                  a.sfb + (static_cast<int64_t>(T.sfb_tile + 1) * a.nkb + kb) * 512, 512,
-                                  &full[stage]);
-                }
                 __syncwarp();
+                mbar_arrive_expect_tx_elect(&full[stage], bytes);
+                tma_load_2d_elect(smem + L::kA + stage * kBM * kBK, &tmap_a, &full[stage], kb * kBK, T.a_row0);
+                tma_load_2d_elect(smem + L::kB + stage * kBBytes, &tmap_b, &full[stage], kb * kBK, T.b_row0);
+                bulk_load_elect(smem + L::kSfa + stage * kSfaBytes,
+                                a.sfa + (static_cast<int64_t>(T.sfa_tile) * a.nkb + kb) * 512, 512, &full[stage]);
+                bulk_load_elect(smem + L::kSfb + stage * kSfbBytes,
+                                a.sfb + (static_cast<int64_t>(T.sfb_tile0) * a.nkb + kb) * 512, 512, &full[stage]);
+                if (sfb1)
+                    bulk_load_elect(smem + L::kSfb + stage * kSfbBytes + 512,
+                                    a.sfb + (static_cast<int64_t>(T.sfb_tile1) * a.nkb + kb) * 512, 512, &full[stage]);
                 ++issued;
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                if (++stage == S) { stage = 0; phase ^= 1u; }
             }
         }
         if (!ok) {
-            // Wait for the copies still in flight (the last min(issued, kStages) fills).
+            // Wait for the copies still in flight (the last min(issued, S) fills).
             int s = stage;
             uint32_t p = phase;
-            for (int i = 0; i < min(issued, kStages); ++i) {
-                if (--s < 0) { s = kStages - 1; p ^= 1u; }
+            for (int i = 0; i < min(issued, S); ++i) {
+                if (--s < 0) { s = S - 1; p ^= 1u; }
                 mbar_wait_drain(&full[s], p, a.timeout_ns);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // Tile j accumulates into TMEM columns [acc_j, acc_j + 256): acc_j = 0 for even j, 240 for odd
-        // j. The two accumulators share columns 240-255, which the epilogue reads first; tile j starts
-        // as soon as those of tile j-1 are drained (by then the epilogue has finished tile j-2). The
-        // scale blocks go to one TMEM slot (columns 496-507): tcgen05 operations issued by one thread
-        // execute in order, so a copy never overtakes the MMAs that read the previous contents.
         int stage = 0;
         uint32_t phase = 0, ovl_phase = 0;
         bool ok = true;
@@ -234,147 +420,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t acc = tmem_base + ((j & 1) ? kAcc1Col : 0u);
             for (int kb = 0; kb < a.nkb; ++kb) {
                 if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    tc_cp_32x128b_warpx4(sfa_t, sdesc_scale_block(smem_u32(smem + kSmemSfa + stage * kSfaBytes)));
-                    tc_cp_32x128b_warpx4(sfb_t, sdesc_scale_block(smem_u32(smem + kSmemSfb + stage * kSfbBytes)));
-                    tc_cp_32x128b_warpx4(sfb_t + 4,
-                                         sdesc_scale_block(smem_u32(smem + kSmemSfb + stage * kSfbBytes + 512)));
-                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(smem + kSmemA + stage * kABytes));
-                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(smem + kSmemB + stage * kBBytes));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        // K-step k: +32 bytes inside the 128-byte swizzled rows; scale byte k.
-                        tc_mma_mxf8(acc, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(kBM, kBN, k),
-                                    sfa_t | (static_cast<uint32_t>(k) << 30), sfb_t | (static_cast<uint32_t>(k) << 30),
-                                    (kb | k) != 0 ? 1u : 0u);
-                    }
-                    tc_commit(&empty[stage]);
-                }
                 __syncwarp();
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                tc_fence_after();
+                tc_cp_elect(sfa_t, sdesc_scale_block(smem_u32(smem + L::kSfa + stage * kSfaBytes)));
+                tc_cp_elect(sfb_t, sdesc_scale_block(smem_u32(smem + L::kSfb + stage * kSfbBytes)));
+                tc_cp_elect(sfb_t + 4, sdesc_scale_block(smem_u32(smem + L::kSfb + stage * kSfbBytes + 512)));
+                const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(smem + L::kA + stage * kBM * kBK));
+                const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(smem + L::kB + stage * kBBytes));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // K-step k: +32 bytes inside the 128-byte swizzled rows; scale byte k.
+                    tc_mma_mxf8_elect(acc, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(kBM, kBN, k),
+                                      sfa_t | (static_cast<uint32_t>(k) << 30), sfb_t | (static_cast<uint32_t>(k) << 30),
+                                      (kb | k) != 0 ? 1u : 0u);
+                }
+                tc_commit_elect(&empty[stage]);
+                if (++stage == S) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(tmem_full);
-            __syncwarp();
+            tc_commit_elect(tmem_full);
         }
-        // Every MMA issued by this thread has completed once `drain` fires.
-        if (lane == 0) tc_commit(drain);
+        // Every MMA issued by this warp has completed once `drain` fires.
         __syncwarp();
+        tc_commit_elect(drain);
         mbar_wait_drain(drain, 0, a.timeout_ns);
     } else {
         // ---------------- epilogue ----------------
-        // Warp w reads TMEM lanes 32 * (w % 4) .. +31 (rows of the tile). The accumulator is released
-        // as soon as its last columns are in registers; rows leave through a per-warp swizzled
-        // staging buffer and a TMA store (32 rows x 128 bytes per store), or, for rows that a TMA
-        // box must not cover (a grouped tile's rows past its group) or unaligned outputs, through
-        // direct masked stores.
         const int q = warp & 3;
-        const int row_local = q * 32 + lane;
-        uint8_t* stage = smem + kSmemStage + (warp - 2) * kStageBytes;
-        const uint32_t stage_row = smem_u32(stage) + lane * 128;
-        const uint32_t swz = static_cast<uint32_t>(lane & 7);
+        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
+        const uint32_t ovl_addr = smem_u32(ovl_free);
         uint32_t full_phase = 0;
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-            const Tile T = decode_tile<GROUPED>(t, a, off, pm);
+            const Tile T = decode_tile1<GROUPED>(t, a, off, pm);
             if (!mbar_wait(tmem_full, full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
-            const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
-            const bool row_ok = row_local < T.rows_valid;
-            const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
-            const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-            const bool acc1 = (j & 1) != 0;
-            const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
-            // The shared columns first (tile columns 240..255 of accumulator 0, 0..15 of accumulator
-            // 1); once every epilogue thread has them, the next tile's MMAs may start.
-            uint32_t ov[16];
-            tc_ld_32x32b_x16(lanes + kOvlCol, ov);
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(ovl_free);
-            // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of this
-            // warp's 32 rows.
-            auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
-                if (col0 >= a.N) return;
-                if (use_tma) {
-                    if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
-                    __syncwarp();
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        st_shared_v4(stage_row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1],
-                                     p[4 * i + 2], p[4 * i + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmap_c, stage, col0, T.a_row0 + q * 32);
-                        bulk_commit_group();
-                    }
-                } else if (row_ok) {
-                    const int ncols = min(cols, a.N - col0);
-                    if (ncols == cols && a.vec_store) {
-                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.c) +
-                                                             (crow * a.ldc + col0) * (a.out_bf16 ? 2 : 4));
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                    } else if (a.out_bf16) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
-#pragma unroll
-                        for (int i = 0; i < 64; ++i)
-                            if (i < ncols) dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
-                    } else {
-                        float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < ncols) dst[i] = __uint_as_float(p[i]);
-                    }
-                }
-            };
-            // Columns [c * 16, c * 16 + 32) for even c: from the shared columns already in `ov` where
-            // they fall there, else from TMEM.
-            auto fetch32 = [&](int c, uint32_t(&p)[32]) {
-                const bool lo_shared = acc1 && c == 0;          // tile columns 0..15 of accumulator 1
-                const bool hi_shared = !acc1 && c == 14;        // tile columns 240..255 of accumulator 0
-                if (lo_shared || hi_shared) {
-                    uint32_t r[16];
-                    tc_ld_32x32b_x16(tq + (lo_shared ? 16u : 224u), r);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        p[i] = lo_shared ? ov[i] : r[i];
-                        p[16 + i] = lo_shared ? r[i] : ov[i];
-                    }
-                } else {
-                    tc_ld_32x32b_x32(tq + c * 16, p);
-                    tc_wait_ld();
-                }
-            };
-            if (a.out_bf16) {
-                uint32_t pk[4][32];                          // the row's 256 columns, packed BF16
-#pragma unroll
-                for (int c = 0; c < 16; c += 2) {
-                    uint32_t r[32];
-                    fetch32(c, r);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                        pk[c >> 2][((c >> 1) & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                }
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) emit(pk[ch], T.n0 + ch * 64, 64);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 16; c += 2) {
-                    uint32_t p[32];
-                    fetch32(c, p);
-                    emit(p, T.n0 + c * 16, 32);
-                }
-            }
+            epilogue_tile<GROUPED>(a, &tmap_c, T, tmem_base, (j & 1) != 0, stage, ovl_addr, q, lane);
         }
-        if (lane == 0) bulk_wait_group<0>();                 // every TMA store of this warp complete
+        if (lane == 0) bulk_wait_group<0>();     // every TMA store of this warp complete
         __syncwarp();
     }
 
@@ -383,6 +467,175 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// CTA-pair kernel: 256 x 256 tiles, cluster of 2 (launched with cluster dimension 2).
+// ---------------------------------------------------------------------------------------------
+constexpr uint32_t kPairStageBytes = kBM * kBK + (kBN / 2) * kBK + kSfaBytes + kSfbBytes;   // per CTA
+
+template <bool GROUPED>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_sfa,
+                        const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs a) {
+    using L = typename std::conditional<GROUPED, SmemPairGrouped, SmemPairDense>::type;
+    constexpr int S = GROUPED ? kStagesPairGrouped : kStagesPairDense;
+    constexpr int kBRows = kBN / 2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // used in the leader CTA only
+    uint64_t* empty = full + S;
+    uint64_t* tmem_full = empty + S;
+    uint64_t* ovl_free = tmem_full + 1;     // leader only: both CTAs' epilogues drained the shared columns
+    uint64_t* drain = ovl_free + 1;
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    int32_t* off = reinterpret_cast<int32_t*>(smem + L::kGroups);
+    int32_t* pm128 = off + (kMaxGroups + 1);
+    int32_t* pm256 = pm128 + (kMaxGroups + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(ovl_free, 8);             // one arrive per epilogue warp of both CTAs
+        mbar_init(drain, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+        prefetch_tensormap(&tmap_sfa);
+        prefetch_tensormap(&tmap_sfb);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_base_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    int tiles;
+    if constexpr (GROUPED)
+        tiles = setup_groups(a, off, pm128, pm256, a.tiles_n);
+    else
+        tiles = a.tiles_m * a.tiles_n;
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                         // both CTAs' barriers initialized before any remote signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs; completions counted in the leader) ----------------
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int t = pair; t < tiles && ok; t += npairs) {
+            const Tile T = decode_tile_pair<GROUPED>(t, rank, a, off, pm128, pm256);
+            for (int kb = 0; kb < a.nkb; ++kb) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
+                __syncwarp();
+                const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                if (leader) mbar_arrive_expect_tx_elect(&full[stage], 2 * kPairStageBytes);
+                tma_load_2d_pair_elect(smem + L::kA + stage * kBM * kBK, &tmap_a, fb, kb * kBK, T.a_row0);
+                tma_load_2d_pair_elect(smem + L::kB + stage * kBRows * kBK, &tmap_b, fb, kb * kBK, T.b_row0);
+                // Scale blocks: the layout viewed as rows of 256 bytes, one block = 2 rows.
+                tma_load_2d_pair_elect(smem + L::kSfa + stage * kSfaBytes, &tmap_sfa, fb, 0,
+                                       2 * (T.sfa_tile * a.nkb + kb));
+                tma_load_2d_pair_elect(smem + L::kSfb + stage * kSfbBytes, &tmap_sfb, fb, 0,
+                                       2 * (T.sfb_tile0 * a.nkb + kb));
+                tma_load_2d_pair_elect(smem + L::kSfb + stage * kSfbBytes + 512, &tmap_sfb, fb, 0,
+                                       2 * (T.sfb_tile1 * a.nkb + kb));
+                ++issued;
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (!ok && leader) {
+            // Wait for the copies still in flight (both CTAs' loads count on the leader's barriers).
+            int s = stage;
+            uint32_t p = phase;
+            for (int i = 0; i < min(issued, S); ++i) {
+                if (--s < 0) { s = S - 1; p ^= 1u; }
+                mbar_wait_drain(&full[s], p, a.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        if (leader) {
+            // ---------------- MMA issuer (leader CTA, for both) ----------------
+            int stage = 0;
+            uint32_t phase = 0, ovl_phase = 0;
+            bool ok = true;
+            const uint32_t sfa_t = tmem_base + kSfCol;
+            const uint32_t sfb_t = sfa_t + 4;
+            int j = 0;
+            for (int t = pair; t < tiles && ok; t += npairs, ++j) {
+                if (j > 0) {
+                    if (!mbar_wait(ovl_free, ovl_phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
+                    ovl_phase ^= 1u;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem_base + ((j & 1) ? kAcc1Col : 0u);
+                for (int kb = 0; kb < a.nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
+                    __syncwarp();
+                    tc_fence_after();
+                    tc_cp_pair_elect(sfa_t, sdesc_scale_block(smem_u32(smem + L::kSfa + stage * kSfaBytes)));
+                    tc_cp_pair_elect(sfb_t, sdesc_scale_block(smem_u32(smem + L::kSfb + stage * kSfbBytes)));
+                    tc_cp_pair_elect(sfb_t + 4, sdesc_scale_block(smem_u32(smem + L::kSfb + stage * kSfbBytes + 512)));
+                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(smem + L::kA + stage * kBM * kBK));
+                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(smem + L::kB + stage * kBRows * kBK));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        tc_mma_mxf8_pair_elect(acc, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(2 * kBM, kBN, k),
+                                               sfa_t | (static_cast<uint32_t>(k) << 30),
+                                               sfb_t | (static_cast<uint32_t>(k) << 30), (kb | k) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair_elect(&empty[stage], 0x3);     // both CTAs' stage is free again
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair_elect(tmem_full, 0x3);
+            }
+            __syncwarp();
+            tc_commit_pair_elect(drain, 0x1);
+            mbar_wait_drain(drain, 0, a.timeout_ns);
+        }
+    } else {
+        // ---------------- epilogue (both CTAs) ----------------
+        const int q = warp & 3;
+        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
+        const uint32_t ovl_addr = mapa_shared(smem_u32(ovl_free), 0);
+        uint32_t full_phase = 0;
+        int j = 0;
+        for (int t = pair; t < tiles; t += npairs, ++j) {
+            const Tile T = decode_tile_pair<GROUPED>(t, rank, a, off, pm128, pm256);
+            if (!mbar_wait(tmem_full, full_phase, abort, a.err, a.timeout_ns)) break;
+            full_phase ^= 1u;
+            tc_fence_after();
+            epilogue_tile<GROUPED>(a, &tmap_c, T, tmem_base, (j & 1) != 0, stage, ovl_addr, q, lane);
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+
+    // Neither CTA leaves (or frees TMEM) while the pair still has MMAs, copies or signals in flight.
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 

@@ -47,8 +47,34 @@ struct DeviceInfo {
     uint32_t* status = nullptr;
     int quant_blocks_per_sm[4] = {0, 0, 0, 0};
     int ge_blocks_per_sm = 1;
+    int pair_clusters[2] = {0, 0};    // co-resident 2-CTA clusters of the pair GEMM (dense, grouped)
     bool ok = false;
 };
+
+// Clusters of 2 CTAs of `kernel` that fit on the device at once (falls back to SMs / 2).
+template <class K>
+int max_pair_clusters(K kernel, int smem, int sms) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = sms / 2;
+    }
+    return n;
+}
+
+// GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
+std::atomic<int> g_gemm_variant{0};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -93,8 +119,14 @@ const DeviceInfo* device_info() {
         if (cudaFuncSetAttribute(mx_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemDense) != cudaSuccess ||
             cudaFuncSetAttribute(mx_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmSmemGrouped) != cudaSuccess)
+                                 kGemmSmemGrouped) != cudaSuccess ||
+            cudaFuncSetAttribute(mx_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmPairSmemDense) != cudaSuccess ||
+            cudaFuncSetAttribute(mx_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmPairSmemGrouped) != cudaSuccess)
             return nullptr;
+        d.pair_clusters[0] = max_pair_clusters(mx_gemm_pair_kernel<false>, kGemmPairSmemDense, d.sms);
+        d.pair_clusters[1] = max_pair_clusters(mx_gemm_pair_kernel<true>, kGemmPairSmemGrouped, d.sms);
         d.ok = true;
     }
     return &d;
@@ -179,6 +211,43 @@ mx_status gemm_checks(const void* qa, const void* sa, const void* qb, const void
 int vector_store_ok(const void* c, int64_t ld_c, mx_out_dtype dt) {
     const int64_t esz = dt == MX_OUT_BF16 ? 2 : 4;
     return aligned16(c) && (ld_c * esz) % 16 == 0;
+}
+
+// Tensor map over a tensor-core scale layout of `blocks` 512-byte blocks, viewed as rows of 256
+// bytes: one block is a 2-row box (loaded by the CTA-pair GEMM through TMA so that the peer CTA's
+// copies count on the leader's barrier).
+bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t blocks) {
+    if (!encode_fn()) return false;
+    const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(2 * blocks)};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {256, 2};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launches the CTA-pair GEMM with a cluster dimension of 2.
+template <bool GROUPED>
+mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                      const CUtensorMap& tsa, const CUtensorMap& tsb, const GemmArgs& a, mx_stream stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = GROUPED ? kGemmPairSmemGrouped : kGemmPairSmemDense;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<GROUPED>, ta, tb, tc, tsa, tsb, a) != cudaSuccess) {
+        cudaGetLastError();
+        return MX_ERR_CUDA;
+    }
+    return launched();
 }
 
 }  // namespace
@@ -443,8 +512,7 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    CUtensorMap ta, tb;
-    if (!make_tmap(&ta, qa, K, M, kBK, kBM) || !make_tmap(&tb, qb, K, N, kBK, kBN)) return MX_ERR_CUDA;
+    const bool pair = g_gemm_variant.load() == 0;
     GemmArgs a{};
     a.sfa = sa_swz;
     a.sfb = sb_swz;
@@ -454,18 +522,29 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     a.N = static_cast<int>(N);
     a.K = static_cast<int>(K);
     a.nkb = static_cast<int>(ceil_div(K, kBK));
-    a.tiles_m = static_cast<int>(ceil_div(M, kBM));
+    a.tiles_m = static_cast<int>(ceil_div(M, pair ? 2 * kBM : kBM));
     a.tiles_n = static_cast<int>(ceil_div(N, kBN));
+    a.sfa_tiles = static_cast<int>(ceil_div(M, 128));
     a.out_bf16 = out_dtype == MX_OUT_BF16;
     a.vec_store = vector_store_ok(c, ld_c, out_dtype);
-    CUtensorMap tc;
-    a.tma_store = make_tmap_out(&tc, c, M, N, ld_c, out_dtype);
     a.G = 1;
     a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
     a.row_offsets = nullptr;
     a.err = d->status;
     a.timeout_ns = g_timeout_ns.load();
+    CUtensorMap ta, tb, tc;
+    a.tma_store = make_tmap_out(&tc, c, M, N, ld_c, out_dtype);
     const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
+    if (pair) {
+        CUtensorMap tsa, tsb;
+        if (!make_tmap(&ta, qa, K, M, kBK, kBM) || !make_tmap(&tb, qb, K, N, kBK, kBN / 2) ||
+            !make_tmap_sf(&tsa, sa_swz, int64_t(a.sfa_tiles) * a.nkb) ||
+            !make_tmap_sf(&tsb, sb_swz, int64_t(a.n_rowtiles) * a.nkb))
+            return MX_ERR_CUDA;
+        const int pairs = static_cast<int>(std::min<int64_t>(tiles, d->pair_clusters[0]));
+        return launch_pair<false>(pairs, ta, tb, tc, tsa, tsb, a, stream);
+    }
+    if (!make_tmap(&ta, qa, K, M, kBK, kBM) || !make_tmap(&tb, qb, K, N, kBK, kBN)) return MX_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, d->sms));
     mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, tc, a);
     return launched();
@@ -484,9 +563,7 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    CUtensorMap ta, tb;
-    if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN))
-        return MX_ERR_CUDA;
+    const bool pair = g_gemm_variant.load() == 0;
     GemmArgs a{};
     a.sfa = sa_swz;
     a.sfb = sb_swz;
@@ -498,20 +575,36 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     a.nkb = static_cast<int>(ceil_div(K, kBK));
     a.tiles_m = 0;
     a.tiles_n = static_cast<int>(ceil_div(N, kBN));
+    a.sfa_tiles = 0;
     a.out_bf16 = out_dtype == MX_OUT_BF16;
     a.vec_store = vector_store_ok(c, ld_c, out_dtype);
-    CUtensorMap tc;
-    a.tma_store = make_tmap_out(&tc, c, total_rows, N, ld_c, out_dtype);
     a.G = static_cast<int>(G);
     a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
     a.row_offsets = row_offsets_dev;
     a.err = d->status;
     a.timeout_ns = g_timeout_ns.load();
+    CUtensorMap ta, tb, tc;
+    a.tma_store = make_tmap_out(&tc, c, total_rows, N, ld_c, out_dtype);
+    if (pair) {
+        // Upper bounds: every group adds at most one partial 256-row tile, one partial 128-row scale tile.
+        const int64_t max_tiles = (ceil_div(total_rows, 2 * kBM) + G) * a.tiles_n;
+        CUtensorMap tsa, tsb;
+        if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN / 2) ||
+            !make_tmap_sf(&tsa, sa_swz, (ceil_div(total_rows, 128) + G) * a.nkb) ||
+            !make_tmap_sf(&tsb, sb_swz, G * a.n_rowtiles * a.nkb))
+            return MX_ERR_CUDA;
+        const int pairs = static_cast<int>(std::min<int64_t>(max_tiles, d->pair_clusters[1]));
+        return launch_pair<true>(pairs, ta, tb, tc, tsa, tsb, a, stream);
+    }
+    if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN))
+        return MX_ERR_CUDA;
     // Upper bound on tiles: every group adds at most one partial 128-row tile.
     const int64_t max_tiles = (ceil_div(total_rows, kBM) + G) * a.tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, d->sms));
     mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, tc, a);
     return launched();
 }
+
+void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
 
 }  // extern "C"

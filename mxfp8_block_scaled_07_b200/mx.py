@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.mx_device_error.restype = I32
     L.mx_set_wait_timeout_ns.argtypes = [U64]
     L.mx_set_wait_timeout_ns.restype = None
+    L.mx_set_gemm_variant.argtypes = [I32]
+    L.mx_set_gemm_variant.restype = None
     L.mx_diag_expired_wait.argtypes = [P]
     L.mx_diag_expired_wait.restype = I32
     _lib = L
@@ -250,3 +252,11 @@ def device_error() -> int:
 
 def set_wait_timeout_ns(ns: int):
     lib().mx_set_wait_timeout_ns(int(ns))
+
+
+GEMM_PAIR, GEMM_SINGLE = 0, 1
+
+
+def set_gemm_variant(variant: int):
+    """0: CTA-pair GEMM kernel (default); 1: single-CTA kernel."""
+    lib().mx_set_gemm_variant(int(variant))

@@ -27,3 +27,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=[0, 1], ids=["pair", "single"])
+def gemm_variant(request):
+    """Runs a GEMM test with the CTA-pair kernel (0, the default) and the single-CTA kernel (1)."""
+    from mxfp8_block_scaled_07_b200 import mx
+
+    mx.set_gemm_variant(request.param)
+    yield request.param
+    mx.set_gemm_variant(0)

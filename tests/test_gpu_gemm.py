@@ -32,22 +32,22 @@ def check_case(A, B, out_dtype, what):
     return assert_gemm_close(to_np(c.float()), ref, abs_sum, out_dtype == torch.bfloat16, what)
 
 
-def test_pr1_full_fp32():
+def test_pr1_full_fp32(gemm_variant):
     A, B = synth.pr1_inputs()
     check_case(A, B, torch.float32, "PR1 256x128x512")
 
 
 @pytest.mark.parametrize("mnk", [(1, 1, 32), (128, 256, 128), (130, 300, 160), (256, 512, 1024), (129, 257, 4160),
-                                 (384, 768, 544), (77, 136, 2048)])
+                                 (384, 768, 544), (77, 136, 2048), (520, 1024, 256), (1000, 600, 640)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_ragged_shapes(mnk, out_dtype):
+def test_ragged_shapes(mnk, out_dtype, gemm_variant):
     M, N, K = mnk
     A = synth.normal_bf16((M, K), seed=M + 3, outlier_frac=0.01, outlier_scale=100.0)
     B = synth.normal_bf16((N, K), std=0.02, seed=N + 5, outlier_frac=0.001, outlier_scale=50.0)
     check_case(A, B, out_dtype, f"{M}x{N}x{K}")
 
 
-def test_identity_like_b_selects_columns_of_a():
+def test_identity_like_b_selects_columns_of_a(gemm_variant):
     # B = rows of the identity (scaled by powers of two) picks single K-columns of A exactly.
     M, K = 160, 256
     A = synth.normal_bf16((M, K), seed=11)
@@ -63,7 +63,7 @@ def test_identity_like_b_selects_columns_of_a():
     assert np.array_equal(to_np(c).astype(np.float64), expect)
 
 
-def test_out_leading_dimension_and_untouched_padding():
+def test_out_leading_dimension_and_untouched_padding(gemm_variant):
     M, N, K = 200, 264, 320
     A = synth.normal_bf16((M, K), seed=21)
     B = synth.normal_bf16((N, K), seed=22)

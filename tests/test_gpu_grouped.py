@@ -52,8 +52,8 @@ def grouped_case(counts, N, K, out_dtype, seed=0, device_inputs=None):
 
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_grouped_small_ragged_with_empty_groups(out_dtype):
-    counts = [0, 5, 128, 129, 300, 0, 1, 64]
+def test_grouped_small_ragged_with_empty_groups(out_dtype, gemm_variant):
+    counts = [0, 5, 128, 129, 300, 0, 1, 64, 256, 257, 511, 2]
     N, K = 384, 256
     X, W, off, c = grouped_case(counts, N, K, out_dtype, seed=3)
     qx, sx = oracle.quantize_rowwise(X)
@@ -62,7 +62,7 @@ def test_grouped_small_ragged_with_empty_groups(out_dtype):
     assert_gemm_close(to_np(c.float()), ref, abs_sum, out_dtype == torch.bfloat16, "grouped small")
 
 
-def test_grouped_bad_offsets_set_device_error_and_write_nothing():
+def test_grouped_bad_offsets_set_device_error_and_write_nothing(gemm_variant):
     counts = [64, 64]
     N, K = 256, 128
     X = synth.normal_bf16((128, K), seed=1).cuda()
