@@ -15,8 +15,9 @@
 //     both. Per SM this halves B traffic and the scale-copy work per FLOP against one CTA alone.
 //   mx_gemm_kernel: one CTA computes a 128 x 256 tile with cta_group::1 MMAs.
 //
-// Roles (192 threads): warp 0 TMA producer (A/B tiles with the 128-byte swizzle, scale blocks);
-// warp 1 TMEM owner and MMA issuer; warps 2-5 epilogue (warp w reads TMEM lanes 32 * (w % 4)).
+// Roles (320 threads): warp 0 TMA producer (A/B tiles with the 128-byte swizzle, scale blocks);
+// warp 1 TMEM owner and MMA issuer; warps 2-9 epilogue in two groups of four (warp w reads TMEM
+// lanes 32 * (w % 4); group (w - 2) / 4 drains one accumulator, i.e. every other tile).
 // TMEM: two accumulators overlapping in 16 columns ([0, 256) and [240, 496)) and one scale slot
 // ([496, 508)): the epilogue drains the shared columns first, so the next tile's MMAs start while
 // the rest of the previous tile is still being read out. tcgen05 operations issued by one thread
@@ -39,7 +40,8 @@ constexpr int kBN = 256;            // columns of C per tile
 constexpr int kBK = 128;            // bytes of K per stage (= one 128-byte swizzle row)
 constexpr int kSfaBytes = 512;
 constexpr int kSfbBytes = 1024;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;          // two groups of four, one warp per TMEM lane quadrant each
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 1024;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns (x 128 lanes, 32-bit): accumulator 0 = [0, 256), accumulator 1 = [240, 496) (the two
@@ -49,9 +51,12 @@ constexpr uint32_t kOvlCol = 240;
 constexpr uint32_t kSfCol = 496;
 constexpr int kStageBytes = 32 * 128;  // epilogue staging per warp: 32 rows x 128 bytes (TMA-store box)
 
-// Shared-memory layout of one kernel configuration. B_ROWS: rows of B per CTA and stage.
-template <int STAGES, int B_ROWS, int GROUP_ARRAYS>
+// Shared-memory layout of one kernel configuration. B_ROWS: rows of B per CTA and stage; BOXES:
+// epilogue staging boxes per warp (TMA stores in flight per warp).
+template <int STAGES, int B_ROWS, int GROUP_ARRAYS, int BOXES>
 struct GemmSmem {
+    static constexpr int kStages = STAGES;
+    static constexpr int kBoxes = BOXES;
     static constexpr int kA = 0;
     static constexpr int kB = kA + STAGES * kBM * kBK;
     static constexpr int kSfa = kB + STAGES * B_ROWS * kBK;
@@ -60,23 +65,21 @@ struct GemmSmem {
     // applies is a function of the address bits 7-9.
     static constexpr int kStage = (kSfb + STAGES * kSfbBytes + 1023) / 1024 * 1024;
     static_assert(kA % 1024 == 0 && kB % 1024 == 0 && kStage % 1024 == 0, "swizzled buffers 1024-aligned");
-    static constexpr int kBar = kStage + 4 * kStageBytes;
-    static constexpr int kMisc = kBar + (2 * STAGES + 3) * 8;
+    static constexpr int kBar = kStage + kEpiWarps * BOXES * kStageBytes;
+    static constexpr int kMisc = kBar + (2 * STAGES + 6) * 8;
     static constexpr int kGroups = (kMisc + 16 + 15) / 16 * 16;
     static constexpr int kBytes = kGroups + GROUP_ARRAYS * (kMaxGroups + 1) * 4 + 1024;   // + alignment slack
 };
-constexpr int kStages1 = 4;                 // single-CTA kernel
-constexpr int kStagesPairDense = 6;         // pair kernel
-constexpr int kStagesPairGrouped = 5;
-using Smem1Dense = GemmSmem<kStages1, kBN, 0>;
-using Smem1Grouped = GemmSmem<kStages1, kBN, 2>;
-using SmemPairDense = GemmSmem<kStagesPairDense, kBN / 2, 0>;
-using SmemPairGrouped = GemmSmem<kStagesPairGrouped, kBN / 2, 3>;
+using Smem1Dense = GemmSmem<3, kBN, 0, 2>;                 // single-CTA kernel
+using Smem1Grouped = GemmSmem<3, kBN, 2, 2>;
+using SmemPairDense = GemmSmem<5, kBN / 2, 0, 1>;          // pair kernel
+using SmemPairGrouped = GemmSmem<4, kBN / 2, 3, 2>;
 constexpr int kGemmSmemDense = Smem1Dense::kBytes;
 constexpr int kGemmSmemGrouped = Smem1Grouped::kBytes;
 constexpr int kGemmPairSmemDense = SmemPairDense::kBytes;
 constexpr int kGemmPairSmemGrouped = SmemPairGrouped::kBytes;
-static_assert(kGemmPairSmemDense <= 232448 && kGemmPairSmemGrouped <= 232448 && kGemmSmemGrouped <= 232448,
+static_assert(kGemmPairSmemDense <= 232448 && kGemmPairSmemGrouped <= 232448 && kGemmSmemGrouped <= 232448 &&
+                  kGemmSmemDense <= 232448,
               "shared memory per CTA");
 
 struct GemmArgs {
@@ -179,16 +182,20 @@ __device__ __forceinline__ Tile decode_tile_pair(int t, int rank, const GemmArgs
     return T;
 }
 
-// Reads the fp32 accumulator of one tile (this warp's 32 TMEM lanes = 32 rows) and writes C.
-// The columns shared by the two accumulators are read first; then one arrive per warp on the
-// `ovl_free` barrier (shared::cluster address) tells the MMA issuer it may start the next tile.
-// Rows leave through the warp's swizzled staging buffer and a TMA store (32 rows x 128 bytes), or,
-// where a TMA box must not go (a grouped tile's rows past its group) or the output is not aligned
-// for TMA, through direct masked stores.
-template <bool GROUPED>
+// Drains the fp32 accumulator of one tile (this warp's 32 TMEM lanes = 32 rows) and writes C.
+// Two epilogue groups of four warps (one warp per TMEM lane quadrant) take the tiles in turn, group
+// g the tiles in accumulator g, so a group that is still storing one tile never delays the drain of
+// the next. The 16 columns the two accumulators share are read first and released with one arrive
+// per warp on `ovl_free`; the accumulator itself is released (`acc_empty`) once the last TMEM load
+// of the tile has landed, before the last store.
+// Rows leave through the warp's BOXES swizzled staging boxes (32 rows x 128 bytes each, used
+// round-robin; `stores` counts this warp's TMA stores across tiles) and TMA stores, or, where a TMA
+// box must not go (a grouped tile's rows past its group) or the output is not aligned for TMA,
+// through direct masked stores. Barrier addresses are shared::cluster addresses.
+template <bool GROUPED, int BOXES>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorMap* tmap_c, const Tile& T,
-                                              uint32_t tmem_base, bool acc1, uint8_t* stage, uint32_t ovl_free_addr,
-                                              int q, int lane) {
+                                              uint32_t tmem_base, bool acc1, uint8_t* stage, uint32_t& stores,
+                                              uint32_t ovl_free_addr, uint32_t acc_empty_addr, int q, int lane) {
     const int row_local = q * 32 + lane;
     const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
     const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
@@ -196,12 +203,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
     const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
     const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
-    const uint32_t stage_row = smem_u32(stage) + lane * 128;
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
 
     uint32_t ov[16];                     // tile columns 240..255 of accumulator 0, 0..15 of accumulator 1
     tc_ld_32x32b_x16(lanes + kOvlCol, ov);
-    tc_wait_ld();
+    tc_wait_ld_regs(ov);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
@@ -210,18 +216,22 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
     auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
         if (col0 >= a.N) return;
         if (use_tma) {
-            if (lane == 0) bulk_wait_group_read<0>();   // staging buffer no longer read
+            uint8_t* box = stage + (stores % BOXES) * kStageBytes;
+            // The box's previous store has read it: at most BOXES - 1 younger stores still reading.
+            if (lane == 0) bulk_wait_group_read<BOXES - 1>();
             __syncwarp();
+            const uint32_t row = smem_u32(box) + lane * 128;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                st_shared_v4(stage_row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1], p[4 * i + 2],
+                st_shared_v4(row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1], p[4 * i + 2],
                              p[4 * i + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_store_2d(tmap_c, stage, col0, T.a_row0 + q * 32);
+                tma_store_2d(tmap_c, box, col0, T.a_row0 + q * 32);
                 bulk_commit_group();
             }
+            ++stores;
         } else if (row_ok) {
             const int ncols = min(cols, a.N - col0);
             if (ncols == cols && a.vec_store) {
@@ -242,45 +252,71 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
             }
         }
     };
-    // Tile columns [c * 16, c * 16 + 32) for even c: from `ov` where they are the shared columns,
-    // else from TMEM.
-    auto fetch32 = [&](int c, uint32_t(&p)[32]) {
-        const bool lo_shared = acc1 && c == 0;
-        const bool hi_shared = !acc1 && c == 14;
-        if (lo_shared || hi_shared) {
-            uint32_t r[16];
-            tc_ld_32x32b_x16(tq + (lo_shared ? 16u : 224u), r);
-            tc_wait_ld();
+    // Issues the TMEM loads of tile columns [32 c, 32 c + 32) into p; the shared columns come from `ov`.
+    // The caller waits (tc_wait_ld_regs) before reading p.
+    auto load32 = [&](int c, uint32_t(&p)[32]) {
+        if (acc1 && c == 0) {
+            tc_ld_32x32b_x16(tq + 16u, *reinterpret_cast<uint32_t(*)[16]>(&p[16]));
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                p[i] = lo_shared ? ov[i] : r[i];
-                p[16 + i] = lo_shared ? r[i] : ov[i];
-            }
+            for (int i = 0; i < 16; ++i) p[i] = ov[i];
+        } else if (!acc1 && c == 7) {
+            tc_ld_32x32b_x16(tq + 224u, *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[16 + i] = ov[i];
         } else {
-            tc_ld_32x32b_x32(tq + c * 16, p);
-            tc_wait_ld();
+            tc_ld_32x32b_x32(tq + 32u * c, p);
+        }
+    };
+    auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_addr);
+    };
+    auto pack = [&](const uint32_t(&r)[64], uint32_t(&pk)[32]) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            pk[i] = *reinterpret_cast<const uint32_t*>(&v);
         }
     };
     if (a.out_bf16) {
-        uint32_t pk[4][32];                  // the row's 256 columns, packed BF16
+        // Four 64-column pieces; the next piece's TMEM loads are in flight while the current one is
+        // stored, and the accumulator is released as soon as the last piece is in registers.
+        uint32_t raw[64], pa[32], pb[32];
+        load32(0, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
+        load32(1, *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
+        tc_wait_ld_regs(raw);
+        pack(raw, pa);
 #pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-            uint32_t r[32];
-            fetch32(c, r);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                pk[c >> 2][((c >> 1) & 1) * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int ch = 0; ch < 4; ++ch) {
+            uint32_t(&cur)[32] = (ch & 1) ? pb : pa;
+            uint32_t(&nxt)[32] = (ch & 1) ? pa : pb;
+            if (ch < 3) {
+                load32(2 * ch + 2, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
+                load32(2 * ch + 3, *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
+            }
+            emit(cur, T.n0 + ch * 64, 64);
+            if (ch < 3) {
+                tc_wait_ld_regs(raw);
+                if (ch == 2) release();
+                pack(raw, nxt);
             }
         }
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) emit(pk[ch], T.n0 + ch * 64, 64);
     } else {
+        // fp32: one 32-column piece at a time, same overlap.
+        uint32_t f0[32], f1[32];
+        load32(0, f0);
+        tc_wait_ld_regs(f0);
 #pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-            uint32_t p[32];
-            fetch32(c, p);
-            emit(p, T.n0 + c * 16, 32);
+        for (int c = 0; c < 8; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? f1 : f0;
+            uint32_t(&nxt)[32] = (c & 1) ? f0 : f1;
+            if (c < 7) load32(c + 1, nxt);
+            emit(cur, T.n0 + c * 32, 32);
+            if (c < 7) {
+                tc_wait_ld_regs(nxt);
+                if (c == 6) release();
+            }
         }
     }
 }
@@ -321,14 +357,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_c, const GemmArgs a) {
     using L = typename std::conditional<GROUPED, Smem1Grouped, Smem1Dense>::type;
-    constexpr int S = kStages1;
+    constexpr int S = L::kStages;
     constexpr int kBBytes = kBN * kBK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
     uint64_t* empty = full + S;
-    uint64_t* tmem_full = empty + S;
-    uint64_t* ovl_free = tmem_full + 1;     // the epilogue has drained the shared accumulator columns
+    uint64_t* tmem_full = empty + S;        // [2]: accumulator g holds a finished tile
+    uint64_t* acc_empty = tmem_full + 2;    // [2]: accumulator g has been read out
+    uint64_t* ovl_free = acc_empty + 2;     // the epilogue has read the shared accumulator columns
     uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -343,8 +380,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(ovl_free, 4);
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&tmem_full[g], 1);
+            mbar_init(&acc_empty[g], kEpiWarps / 2);
+        }
+        mbar_init(ovl_free, kEpiWarps / 2);
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -406,13 +446,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         int stage = 0;
-        uint32_t phase = 0, ovl_phase = 0;
+        uint32_t phase = 0, ovl_phase = 0, empty_phase = 0;
         bool ok = true;
         const uint32_t sfa_t = tmem_base + kSfCol;
         const uint32_t sfb_t = sfa_t + 4;
         int j = 0;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
-            if (j > 0) {
+            if (j > 1) {                    // the accumulator's previous tile has been read out
+                if (!mbar_wait(&acc_empty[j & 1], (empty_phase >> (j & 1)) & 1u, abort, a.err, a.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                empty_phase ^= 1u << (j & 1);
+            }
+            if (j > 0) {                    // the previous tile's shared columns have been read
                 if (!mbar_wait(ovl_free, ovl_phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
                 ovl_phase ^= 1u;
             }
@@ -438,7 +485,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
-            tc_commit_elect(tmem_full);
+            tc_commit_elect(&tmem_full[j & 1]);
         }
         // Every MMA issued by this warp has completed once `drain` fires.
         __syncwarp();
@@ -446,17 +493,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_drain(drain, 0, a.timeout_ns);
     } else {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;
-        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
+        const int q = warp & 3;             // TMEM lane quadrant this warp may access
+        const int g = (warp - 2) >> 2;      // group: drains accumulator g, i.e. every other tile
+        uint8_t* stage = smem + L::kStage + (warp - 2) * L::kBoxes * kStageBytes;
+        uint32_t stores = 0;
         const uint32_t ovl_addr = smem_u32(ovl_free);
+        const uint32_t empty_addr = smem_u32(&acc_empty[g]);
         uint32_t full_phase = 0;
-        int j = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+        for (int t = blockIdx.x + g * gridDim.x; t < tiles; t += 2 * gridDim.x) {
             const Tile T = decode_tile1<GROUPED>(t, a, off, pm);
-            if (!mbar_wait(tmem_full, full_phase, abort, a.err, a.timeout_ns)) break;
+            if (!mbar_wait(&tmem_full[g], full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            epilogue_tile<GROUPED>(a, &tmap_c, T, tmem_base, (j & 1) != 0, stage, ovl_addr, q, lane);
+            epilogue_tile<GROUPED, L::kBoxes>(a, &tmap_c, T, tmem_base, g != 0, stage, stores, ovl_addr,
+                                               empty_addr, q, lane);
         }
         if (lane == 0) bulk_wait_group<0>();     // every TMA store of this warp complete
         __syncwarp();
@@ -481,14 +531,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_sfa,
                         const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs a) {
     using L = typename std::conditional<GROUPED, SmemPairGrouped, SmemPairDense>::type;
-    constexpr int S = GROUPED ? kStagesPairGrouped : kStagesPairDense;
+    constexpr int S = L::kStages;
     constexpr int kBRows = kBN / 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // used in the leader CTA only
     uint64_t* empty = full + S;
-    uint64_t* tmem_full = empty + S;
-    uint64_t* ovl_free = tmem_full + 1;     // leader only: both CTAs' epilogues drained the shared columns
+    uint64_t* tmem_full = empty + S;        // [2]: accumulator g holds a finished tile (both CTAs)
+    uint64_t* acc_empty = tmem_full + 2;    // [2], leader only: accumulator g read out in both CTAs
+    uint64_t* ovl_free = acc_empty + 2;     // leader only: both CTAs' epilogues read the shared columns
     uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -508,8 +559,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(ovl_free, 8);             // one arrive per epilogue warp of both CTAs
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&tmem_full[g], 1);
+            mbar_init(&acc_empty[g], kEpiWarps);    // one arrive per warp of one group in both CTAs
+        }
+        mbar_init(ovl_free, kEpiWarps);
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -574,13 +628,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (leader) {
             // ---------------- MMA issuer (leader CTA, for both) ----------------
             int stage = 0;
-            uint32_t phase = 0, ovl_phase = 0;
+            uint32_t phase = 0, ovl_phase = 0, empty_phase = 0;
             bool ok = true;
             const uint32_t sfa_t = tmem_base + kSfCol;
             const uint32_t sfb_t = sfa_t + 4;
             int j = 0;
             for (int t = pair; t < tiles && ok; t += npairs, ++j) {
-                if (j > 0) {
+                if (j > 1) {                // the accumulator's previous tile has been read out
+                    if (!mbar_wait(&acc_empty[j & 1], (empty_phase >> (j & 1)) & 1u, abort, a.err,
+                                   a.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    empty_phase ^= 1u << (j & 1);
+                }
+                if (j > 0) {                // the previous tile's shared columns have been read
                     if (!mbar_wait(ovl_free, ovl_phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
                     ovl_phase ^= 1u;
                 }
@@ -605,7 +667,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit_pair_elect(tmem_full, 0x3);
+                tc_commit_pair_elect(&tmem_full[j & 1], 0x3);
             }
             __syncwarp();
             tc_commit_pair_elect(drain, 0x1);
@@ -613,17 +675,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ---------------- epilogue (both CTAs) ----------------
-        const int q = warp & 3;
-        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
+        const int q = warp & 3;             // TMEM lane quadrant this warp may access
+        const int g = (warp - 2) >> 2;      // group: drains accumulator g, i.e. every other tile
+        uint8_t* stage = smem + L::kStage + (warp - 2) * L::kBoxes * kStageBytes;
+        uint32_t stores = 0;
         const uint32_t ovl_addr = mapa_shared(smem_u32(ovl_free), 0);
+        const uint32_t empty_addr = mapa_shared(smem_u32(&acc_empty[g]), 0);
         uint32_t full_phase = 0;
-        int j = 0;
-        for (int t = pair; t < tiles; t += npairs, ++j) {
+        for (int t = pair + g * npairs; t < tiles; t += 2 * npairs) {
             const Tile T = decode_tile_pair<GROUPED>(t, rank, a, off, pm128, pm256);
-            if (!mbar_wait(tmem_full, full_phase, abort, a.err, a.timeout_ns)) break;
+            if (!mbar_wait(&tmem_full[g], full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            epilogue_tile<GROUPED>(a, &tmap_c, T, tmem_base, (j & 1) != 0, stage, ovl_addr, q, lane);
+            epilogue_tile<GROUPED, L::kBoxes>(a, &tmap_c, T, tmem_base, g != 0, stage, stores, ovl_addr,
+                                               empty_addr, q, lane);
         }
         if (lane == 0) bulk_wait_group<0>();
         __syncwarp();

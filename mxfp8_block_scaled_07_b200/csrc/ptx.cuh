@@ -172,6 +172,24 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's TMEM loads and ties the destination registers to the wait, so no use of
+// them is scheduled above it.
+template <int N>
+__device__ __forceinline__ void reg_after_wait(uint32_t (&r)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+template <int N>
+__device__ __forceinline__ void tc_wait_ld_regs(uint32_t (&r)[N]) {
+    tc_wait_ld();
+    reg_after_wait(r);
+}
+template <int N>
+__device__ __forceinline__ void tc_wait_ld_regs(uint32_t (&r0)[N], uint32_t (&r1)[N]) {
+    tc_wait_ld();
+    reg_after_wait(r0);
+    reg_after_wait(r1);
+}
 
 // 32 lanes x 32 columns of 32-bit words: thread t of the warp gets lane (base_lane + t), columns
 // [col, col + 32).
