@@ -307,8 +307,9 @@ def sum_over_ranks(pg, value: int) -> int:
 
 
 def traffic_record():
-    """DRAM bytes per launch of the quantize kernel from a committed ncu summary, valid only while
-    the kernel source is unchanged (sha256 of the sources it was measured on)."""
+    """DRAM bytes per element of the multi-tensor quantize launch from a committed ncu summary,
+    valid only while the kernel source is unchanged (sha256 of quantize.cuh, which holds the whole
+    kernel and its device helpers)."""
     import hashlib
 
     p = os.path.join(ROOT, "profiles", "quantize_rowwise_traffic.json")
@@ -318,7 +319,7 @@ def traffic_record():
     except (OSError, ValueError):
         return None
     h = hashlib.sha256()
-    for f in ("quantize.cuh", "ptx.cuh", "libmx.cu"):
+    for f in ("quantize.cuh",):
         with open(os.path.join(ROOT, "mxfp8_block_scaled_07_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     if rec.get("source_sha256") != h.hexdigest():
