@@ -22,7 +22,7 @@
 // ([496, 508)): the epilogue drains the shared columns first, so the next tile's MMAs start while
 // the rest of the previous tile is still being read out. tcgen05 operations issued by one thread
 // execute in order, so a scale copy never overtakes the MMAs that read the slot's previous contents.
-// The epilogue writes through per-warp swizzled staging and TMA stores.
+// The epilogue writes through per-warp swizzled staging and coalesced 16-byte stores.
 //
 // Every mbarrier wait is bounded (globaltimer deadline); on expiry the kernel records an error bit,
 // stops all roles, drains its in-flight copies and MMAs, frees TMEM and returns. No load uses
@@ -49,31 +49,27 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 240;
 constexpr uint32_t kOvlCol = 240;
 constexpr uint32_t kSfCol = 496;
-constexpr int kStageBytes = 32 * 128;  // epilogue staging per warp: 32 rows x 128 bytes (TMA-store box)
+constexpr int kStageBytes = 32 * 128;  // epilogue staging per warp: 32 rows x 128 bytes
 
-// Shared-memory layout of one kernel configuration. B_ROWS: rows of B per CTA and stage; BOXES:
-// epilogue staging boxes per warp (TMA stores in flight per warp).
-template <int STAGES, int B_ROWS, int GROUP_ARRAYS, int BOXES>
+// Shared-memory layout of one kernel configuration. B_ROWS: rows of B per CTA and stage.
+template <int STAGES, int B_ROWS, int GROUP_ARRAYS>
 struct GemmSmem {
     static constexpr int kStages = STAGES;
-    static constexpr int kBoxes = BOXES;
     static constexpr int kA = 0;
     static constexpr int kB = kA + STAGES * kBM * kBK;
     static constexpr int kSfa = kB + STAGES * B_ROWS * kBK;
     static constexpr int kSfb = kSfa + STAGES * kSfaBytes;
-    // The staging buffers must start on a 1024-byte boundary: the 128-byte swizzle the TMA store
-    // applies is a function of the address bits 7-9.
     static constexpr int kStage = (kSfb + STAGES * kSfbBytes + 1023) / 1024 * 1024;
-    static_assert(kA % 1024 == 0 && kB % 1024 == 0 && kStage % 1024 == 0, "swizzled buffers 1024-aligned");
-    static constexpr int kBar = kStage + kEpiWarps * BOXES * kStageBytes;
+    static_assert(kA % 1024 == 0 && kB % 1024 == 0, "swizzled operand buffers 1024-aligned");
+    static constexpr int kBar = kStage + kEpiWarps * kStageBytes;
     static constexpr int kMisc = kBar + (2 * STAGES + 6) * 8;
     static constexpr int kGroups = (kMisc + 16 + 15) / 16 * 16;
     static constexpr int kBytes = kGroups + GROUP_ARRAYS * (kMaxGroups + 1) * 4 + 1024;   // + alignment slack
 };
-using Smem1Dense = GemmSmem<3, kBN, 0, 2>;                 // single-CTA kernel
-using Smem1Grouped = GemmSmem<3, kBN, 2, 2>;
-using SmemPairDense = GemmSmem<5, kBN / 2, 0, 1>;          // pair kernel
-using SmemPairGrouped = GemmSmem<4, kBN / 2, 3, 2>;
+using Smem1Dense = GemmSmem<3, kBN, 0>;                    // single-CTA kernel
+using Smem1Grouped = GemmSmem<3, kBN, 2>;
+using SmemPairDense = GemmSmem<5, kBN / 2, 0>;             // pair kernel
+using SmemPairGrouped = GemmSmem<5, kBN / 2, 3>;
 constexpr int kGemmSmemDense = Smem1Dense::kBytes;
 constexpr int kGemmSmemGrouped = Smem1Grouped::kBytes;
 constexpr int kGemmPairSmemDense = SmemPairDense::kBytes;
@@ -94,8 +90,7 @@ struct GemmArgs {
     int tiles_n;        // 256-column tiles
     int sfa_tiles;      // 128-row tiles in A's scale layout (dense), for clamping
     int out_bf16;
-    int vec_store;      // output rows 16-byte aligned: full 32-column chunks use 16-byte stores
-    int tma_store;      // output written by TMA from swizzled shared-memory staging (tmap_c valid)
+    int vec_store;      // output rows 16-byte aligned: full 16-byte chunks use 16-byte stores
     int G;
     int n_rowtiles;     // ceil(N / 128): scale row-tiles of one B operand
     const int32_t* row_offsets;
@@ -188,19 +183,17 @@ __device__ __forceinline__ Tile decode_tile_pair(int t, int rank, const GemmArgs
 // the next. The 16 columns the two accumulators share are read first and released with one arrive
 // per warp on `ovl_free`; the accumulator itself is released (`acc_empty`) once the last TMEM load
 // of the tile has landed, before the last store.
-// Rows leave through the warp's BOXES swizzled staging boxes (32 rows x 128 bytes each, used
-// round-robin; `stores` counts this warp's TMA stores across tiles) and TMA stores, or, where a TMA
-// box must not go (a grouped tile's rows past its group) or the output is not aligned for TMA,
-// through direct masked stores. Barrier addresses are shared::cluster addresses.
-template <bool GROUPED, int BOXES>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorMap* tmap_c, const Tile& T,
-                                              uint32_t tmem_base, bool acc1, uint8_t* stage, uint32_t& stores,
-                                              uint32_t ovl_free_addr, uint32_t acc_empty_addr, int q, int lane) {
-    const int row_local = q * 32 + lane;
+// Rows leave through the warp's swizzled staging box (32 rows x 128 bytes): each lane writes its
+// row there, then the warp writes the box out row-contiguous with 16-byte stores (8 lanes per row,
+// 4 rows per instruction), masked to the tile's valid rows and to N. The stores go through the
+// load/store path, not TMA: TMA stores share the SM's TMA unit with the operand loads and were
+// measured to slow those down. Barrier addresses are shared::cluster addresses.
+template <bool GROUPED>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, uint32_t tmem_base, bool acc1,
+                                              uint8_t* stage, uint32_t ovl_free_addr, uint32_t acc_empty_addr,
+                                              int q, int lane) {
     const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
-    const bool use_tma = a.tma_store && warp_rows > 0 && (!GROUPED || warp_rows == 32);
-    const bool row_ok = row_local < T.rows_valid;
-    const int64_t crow = static_cast<int64_t>(T.a_row0) + row_local;
+    const int64_t row0 = static_cast<int64_t>(T.a_row0) + q * 32;
     const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
@@ -213,44 +206,45 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
     if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
 
     // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of the 32 rows.
-    auto emit = [&](const uint32_t(&p)[32], int col0, int cols) {
+    const uint32_t box = smem_u32(stage);
+    const int esz = a.out_bf16 ? 2 : 4;
+    const int epc = 16 / esz;                            // elements per 16-byte chunk
+    auto emit = [&](const uint32_t(&p)[32], int col0) {
         if (col0 >= a.N) return;
-        if (use_tma) {
-            uint8_t* box = stage + (stores % BOXES) * kStageBytes;
-            // The box's previous store has read it: at most BOXES - 1 younger stores still reading.
-            if (lane == 0) bulk_wait_group_read<BOXES - 1>();
-            __syncwarp();
-            const uint32_t row = smem_u32(box) + lane * 128;
+        const uint32_t row = box + lane * 128;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                st_shared_v4(row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1], p[4 * i + 2],
-                             p[4 * i + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_2d(tmap_c, box, col0, T.a_row0 + q * 32);
-                bulk_commit_group();
-            }
-            ++stores;
-        } else if (row_ok) {
-            const int ncols = min(cols, a.N - col0);
-            if (ncols == cols && a.vec_store) {
-                uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.c) +
-                                                     (crow * a.ldc + col0) * (a.out_bf16 ? 2 : 4));
+        for (int i = 0; i < 8; ++i)
+            st_shared_v4(row + ((static_cast<uint32_t>(i) ^ swz) << 4), p[4 * i], p[4 * i + 1], p[4 * i + 2],
+                         p[4 * i + 3]);
+        __syncwarp();
+        const int c = lane & 7;                          // this lane's 16-byte chunk of each row
+        const int gc = col0 + c * epc;
+        const int ncols = min(epc, a.N - gc);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-            } else if (a.out_bf16) {
-                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.c) + crow * a.ldc + col0;
+        for (int i = 0; i < 8; ++i) {
+            const int rr = (lane >> 3) + 4 * i;
+            const uint4 v = ld_shared_v4(box + rr * 128 + ((static_cast<uint32_t>(c) ^ (rr & 7)) << 4));
+            if (rr < warp_rows && ncols > 0) {
+                uint8_t* dst = static_cast<uint8_t*>(a.c) + ((row0 + rr) * a.ldc + gc) * esz;
+                if (ncols == epc && a.vec_store) {
+                    st_global_v4(dst, v);
+                } else {
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    if (a.out_bf16) {
+                        uint16_t* d = reinterpret_cast<uint16_t*>(dst);
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (i < ncols) dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(p[i >> 1] >> (16 * (i & 1))));
-            } else {
-                float* dst = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
+                        for (int e = 0; e < 8; ++e)
+                            if (e < ncols) d[e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+                    } else {
+                        uint32_t* d = reinterpret_cast<uint32_t*>(dst);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (i < ncols) dst[i] = __uint_as_float(p[i]);
+                        for (int e = 0; e < 4; ++e)
+                            if (e < ncols) d[e] = w[e];
+                    }
+                }
             }
         }
+        __syncwarp();                                    // the box is free for the next piece
     };
     // Issues the TMEM loads of tile columns [32 c, 32 c + 32) into p; the shared columns come from `ov`.
     // The caller waits (tc_wait_ld_regs) before reading p.
@@ -295,7 +289,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
                 load32(2 * ch + 2, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
                 load32(2 * ch + 3, *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
             }
-            emit(cur, T.n0 + ch * 64, 64);
+            emit(cur, T.n0 + ch * 64);
             if (ch < 3) {
                 tc_wait_ld_regs(raw);
                 if (ch == 2) release();
@@ -312,7 +306,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const CUtensorM
             uint32_t(&cur)[32] = (c & 1) ? f1 : f0;
             uint32_t(&nxt)[32] = (c & 1) ? f0 : f1;
             if (c < 7) load32(c + 1, nxt);
-            emit(cur, T.n0 + c * 32, 32);
+            emit(cur, T.n0 + c * 32);
             if (c < 7) {
                 tc_wait_ld_regs(nxt);
                 if (c == 6) release();
@@ -355,7 +349,7 @@ __device__ __forceinline__ int setup_groups(const GemmArgs& a, int32_t* off, int
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                   const __grid_constant__ CUtensorMap tmap_c, const GemmArgs a) {
+                   const GemmArgs a) {
     using L = typename std::conditional<GROUPED, Smem1Grouped, Smem1Dense>::type;
     constexpr int S = L::kStages;
     constexpr int kBBytes = kBN * kBK;
@@ -495,8 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---------------- epilogue ----------------
         const int q = warp & 3;             // TMEM lane quadrant this warp may access
         const int g = (warp - 2) >> 2;      // group: drains accumulator g, i.e. every other tile
-        uint8_t* stage = smem + L::kStage + (warp - 2) * L::kBoxes * kStageBytes;
-        uint32_t stores = 0;
+        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
         const uint32_t ovl_addr = smem_u32(ovl_free);
         const uint32_t empty_addr = smem_u32(&acc_empty[g]);
         uint32_t full_phase = 0;
@@ -505,11 +498,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait(&tmem_full[g], full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            epilogue_tile<GROUPED, L::kBoxes>(a, &tmap_c, T, tmem_base, g != 0, stage, stores, ovl_addr,
-                                               empty_addr, q, lane);
+            epilogue_tile<GROUPED>(a, T, tmem_base, g != 0, stage, ovl_addr, empty_addr, q, lane);
         }
-        if (lane == 0) bulk_wait_group<0>();     // every TMA store of this warp complete
-        __syncwarp();
     }
 
     tc_fence_before();
@@ -528,8 +518,8 @@ constexpr uint32_t kPairStageBytes = kBM * kBK + (kBN / 2) * kBK + kSfaBytes + k
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                        const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_sfa,
-                        const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                        const GemmArgs a) {
     using L = typename std::conditional<GROUPED, SmemPairGrouped, SmemPairDense>::type;
     constexpr int S = L::kStages;
     constexpr int kBRows = kBN / 2;
@@ -677,8 +667,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---------------- epilogue (both CTAs) ----------------
         const int q = warp & 3;             // TMEM lane quadrant this warp may access
         const int g = (warp - 2) >> 2;      // group: drains accumulator g, i.e. every other tile
-        uint8_t* stage = smem + L::kStage + (warp - 2) * L::kBoxes * kStageBytes;
-        uint32_t stores = 0;
+        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
         const uint32_t ovl_addr = mapa_shared(smem_u32(ovl_free), 0);
         const uint32_t empty_addr = mapa_shared(smem_u32(&acc_empty[g]), 0);
         uint32_t full_phase = 0;
@@ -687,11 +676,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait(&tmem_full[g], full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            epilogue_tile<GROUPED, L::kBoxes>(a, &tmap_c, T, tmem_base, g != 0, stage, stores, ovl_addr,
-                                               empty_addr, q, lane);
+            epilogue_tile<GROUPED>(a, T, tmem_base, g != 0, stage, ovl_addr, empty_addr, q, lane);
         }
-        if (lane == 0) bulk_wait_group<0>();
-        __syncwarp();
     }
 
     // Neither CTA leaves (or frees TMEM) while the pair still has MMAs, copies or signals in flight.

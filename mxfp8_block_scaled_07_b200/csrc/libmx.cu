@@ -172,24 +172,6 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Tensor map for the GEMM output C[rows, N] (row stride ld_c elements) written by the epilogue's
-// TMA stores: 32-row boxes of 128 bytes (64 BF16 or 32 fp32 columns), 128-byte swizzle. Returns
-// false (and the epilogue uses direct stores) when C's base or row stride is not 16-byte aligned.
-bool make_tmap_out(CUtensorMap* map, const void* c, int64_t rows, int64_t N, int64_t ld_c, mx_out_dtype dt) {
-    std::memset(map, 0, sizeof *map);
-    const int64_t esz = dt == MX_OUT_BF16 ? 2 : 4;
-    if (!aligned16(c) || (ld_c * esz) % 16 != 0) return false;
-    if (!encode_fn()) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_c * esz)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32};
-    const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, dt == MX_OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-                    const_cast<void*>(c), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Checks shared by both GEMMs. Sets *empty when there is nothing to compute (then pointers may be
 // null). The output may have any element alignment; 16-byte aligned rows take vector stores.
 mx_status gemm_checks(const void* qa, const void* sa, const void* qb, const void* sb, int64_t M, int64_t N,
@@ -229,8 +211,8 @@ bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t blocks) {
 
 // Launches the CTA-pair GEMM with a cluster dimension of 2.
 template <bool GROUPED>
-mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
-                      const CUtensorMap& tsa, const CUtensorMap& tsb, const GemmArgs& a, mx_stream stream) {
+mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                      const CUtensorMap& tsb, const GemmArgs& a, mx_stream stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -243,7 +225,7 @@ mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<GROUPED>, ta, tb, tc, tsa, tsb, a) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<GROUPED>, ta, tb, tsa, tsb, a) != cudaSuccess) {
         cudaGetLastError();
         return MX_ERR_CUDA;
     }
@@ -532,8 +514,7 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     a.row_offsets = nullptr;
     a.err = d->status;
     a.timeout_ns = g_timeout_ns.load();
-    CUtensorMap ta, tb, tc;
-    a.tma_store = make_tmap_out(&tc, c, M, N, ld_c, out_dtype);
+    CUtensorMap ta, tb;
     const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
     if (pair) {
         CUtensorMap tsa, tsb;
@@ -542,11 +523,11 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
             !make_tmap_sf(&tsb, sb_swz, int64_t(a.n_rowtiles) * a.nkb))
             return MX_ERR_CUDA;
         const int pairs = static_cast<int>(std::min<int64_t>(tiles, d->pair_clusters[0]));
-        return launch_pair<false>(pairs, ta, tb, tc, tsa, tsb, a, stream);
+        return launch_pair<false>(pairs, ta, tb, tsa, tsb, a, stream);
     }
     if (!make_tmap(&ta, qa, K, M, kBK, kBM) || !make_tmap(&tb, qb, K, N, kBK, kBN)) return MX_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, d->sms));
-    mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, tc, a);
+    mx_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemDense, stream>>>(ta, tb, a);
     return launched();
 }
 
@@ -583,8 +564,7 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     a.row_offsets = row_offsets_dev;
     a.err = d->status;
     a.timeout_ns = g_timeout_ns.load();
-    CUtensorMap ta, tb, tc;
-    a.tma_store = make_tmap_out(&tc, c, total_rows, N, ld_c, out_dtype);
+    CUtensorMap ta, tb;
     if (pair) {
         // Upper bounds: every group adds at most one partial 256-row tile, one partial 128-row scale tile.
         const int64_t max_tiles = (ceil_div(total_rows, 2 * kBM) + G) * a.tiles_n;
@@ -594,14 +574,14 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
             !make_tmap_sf(&tsb, sb_swz, G * a.n_rowtiles * a.nkb))
             return MX_ERR_CUDA;
         const int pairs = static_cast<int>(std::min<int64_t>(max_tiles, d->pair_clusters[1]));
-        return launch_pair<true>(pairs, ta, tb, tc, tsa, tsb, a, stream);
+        return launch_pair<true>(pairs, ta, tb, tsa, tsb, a, stream);
     }
     if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN))
         return MX_ERR_CUDA;
     // Upper bound on tiles: every group adds at most one partial 128-row tile.
     const int64_t max_tiles = (ceil_div(total_rows, kBM) + G) * a.tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, d->sms));
-    mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, tc, a);
+    mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, a);
     return launched();
 }
 
