@@ -84,10 +84,10 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn g_encode = nullptr;
 std::once_flag g_encode_once;
 
-template <bool R, bool C>
+template <bool ROW>
 int quant_occupancy() {
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<R, C, kQMaxTensors>, kQThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_rowcol_kernel<ROW, kQMaxTensors>, kQThreads, 0);
     return n > 0 ? n : 1;
 }
 
@@ -111,8 +111,8 @@ const DeviceInfo* device_info() {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1], quantize_rowwise_kernel<kQMaxTensors>,
                                                       kQThreads, 0);
         if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
-        d.quant_blocks_per_sm[2] = quant_occupancy<false, true>();
-        d.quant_blocks_per_sm[3] = quant_occupancy<true, true>();
+        d.quant_blocks_per_sm[2] = quant_occupancy<false>();
+        d.quant_blocks_per_sm[3] = quant_occupancy<true>();
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.ge_blocks_per_sm, grid_equal_kernel<kGeMaxPairs>,
                                                       kGeThreads, 0);
         if (d.ge_blocks_per_sm < 1) d.ge_blocks_per_sm = 1;
@@ -313,6 +313,7 @@ void add_quant_tensor(QuantArgs<NT>& a, const mx_quant_tensor& t) {
     q.tiles_k = static_cast<int32_t>(ceil_div(t.K, kQTile));
     q.vec32 = (reinterpret_cast<uintptr_t>(t.x) % 32 == 0) && (t.ld_x % 16 == 0) &&
               (reinterpret_cast<uintptr_t>(t.q_row) % 32 == 0);
+    q.col_vec32 = reinterpret_cast<uintptr_t>(t.q_col) % 32 == 0;
     q.tile_start = a.total_tiles;
     a.total_tiles += int64_t(q.tiles_m) * q.tiles_k;
 }
@@ -323,11 +324,11 @@ mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceI
     const int which = (row ? 1 : 0) | (col ? 2 : 0);
     const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
     if (row && col)
-        quantize_kernel<true, true, NT><<<grid, kQThreads, 0, stream>>>(a);
+        quantize_rowcol_kernel<true, NT><<<grid, kQThreads, 0, stream>>>(a);
     else if (row)
         quantize_rowwise_kernel<NT><<<grid, kQThreads, 0, stream>>>(a);
     else
-        quantize_kernel<false, true, NT><<<grid, kQThreads, 0, stream>>>(a);
+        quantize_rowcol_kernel<false, NT><<<grid, kQThreads, 0, stream>>>(a);
     return launched();
 }
 

@@ -133,6 +133,7 @@ struct QTensor {
     int64_t tile_start;       // first tile of this tensor in the launch's tile space
     int32_t tiles_m, tiles_k;
     int32_t vec32;            // x rows and q_row 32-byte aligned: 256-bit loads and stores
+    int32_t col_vec32;        // q_col 32-byte aligned: 256-bit stores of the transposed copy
 };
 
 struct Block32 {
@@ -193,187 +194,6 @@ __device__ __forceinline__ TileRef decode_qtile(const QuantArgs<NT>& a, int64_t 
     r.k0 = static_cast<int64_t>(r.kt) * kQTile;
     r.full = (r.m0 + kQTile <= T.M) && (r.k0 + kQTile <= T.K);
     return r;
-}
-
-// Thread tid loads chunk (tid & 15) of rows it * 16 + (tid >> 4), it = 0..7.
-template <int NT>
-__device__ __forceinline__ void load_qtile(const QuantArgs<NT>& a, const TileRef& r, uint4 (&v)[8], int tid) {
-    const QTensor& T = a.t[r.i];
-    const int cc = tid & 15;
-    const uint16_t* base = T.x + (r.m0 + (tid >> 4)) * T.ldx + r.k0 + cc * 8;
-    const int64_t step = 16 * T.ldx;
-    if (r.full) {
-#pragma unroll
-        for (int it = 0; it < 8; ++it) v[it] = ld_stream_v4(base + it * step);
-    } else {
-        const bool kok = r.k0 + cc * 8 < T.K;
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const bool ok = kok && (r.m0 + it * 16 + (tid >> 4) < T.M);
-            v[it] = ok ? ld_stream_v4(base + it * step) : make_uint4(0, 0, 0, 0);
-        }
-    }
-}
-
-template <bool ROW, bool COL, int NT>
-__global__ void __launch_bounds__(kQThreads, 3) quantize_kernel(const __grid_constant__ QuantArgs<NT> a) {
-    __shared__ __align__(16) uint4 tile[COL ? kQTile * 16 : 1];   // 128 rows x 16 chunks of 8 BF16
-    __shared__ __align__(16) uint8_t atom_row[512];
-    __shared__ __align__(16) uint8_t atom_col[512];
-
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
-
-    // Each CTA owns a contiguous range of the tile space: one decode at the start, then the next
-    // tile is found by stepping (tensor, row tile, column tile) without divisions.
-    const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
-    const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
-    const int64_t t_end = min(a.total_tiles, t_begin + per);
-    uint4 cur[8], nxt[8];
-    TileRef rc, rn;
-    if (t_begin < t_end) {
-        rc = decode_qtile(a, t_begin);
-        load_qtile(a, rc, cur, tid);
-    }
-    for (int64_t t = t_begin; t < t_end; ++t) {
-        if (t + 1 < t_end) {
-            rn = rc;
-            if (++rn.kt == a.t[rn.i].tiles_k) {
-                rn.kt = 0;
-                if (++rn.mt == a.t[rn.i].tiles_m) {
-                    rn.mt = 0;
-                    ++rn.i;
-                }
-            }
-            const QTensor& Tn = a.t[rn.i];
-            rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
-            rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
-            rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
-            load_qtile(a, rn, nxt, tid);
-        }
-        const QTensor& T = a.t[rc.i];
-        const int64_t kblocks = T.K / 32;
-
-        if constexpr (COL) {
-#pragma unroll
-            for (int it = 0; it < 8; ++it) tile[(it * 16 + (tid >> 4)) * 16 + (tid & 15)] = cur[it];
-        }
-
-        if constexpr (ROW) {
-            // Four consecutive lanes hold one 32-block (8 BF16 each) of one row.
-            const int cc = tid & 15;
-            const bool kok = rc.k0 + cc * 8 < T.K;
-            uint8_t* qbase = T.q_row + (rc.m0 + (tid >> 4)) * T.K + rc.k0 + cc * 8;
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const int row = it * 16 + (tid >> 4);
-                const bool valid = rc.full || (kok && rc.m0 + row < T.M);
-                const uint4 v = cur[it];
-                uint32_t mx = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)) & 0x7FFF7FFFu;
-                mx = max(mx & 0xFFFFu, mx >> 16);
-                mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-                mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-                const uint32_t s = scale_byte_from_amax(mx);
-                if (valid) *reinterpret_cast<uint2*>(qbase + it * 16 * T.K) = encode_chunk(v, s);
-                if ((lane & 3) == 0)
-                    atom_row[(row & 31) * 16 + (row >> 5) * 4 + (cc >> 2)] = valid ? static_cast<uint8_t>(s) : 0;
-            }
-        }
-
-        if constexpr (COL) {
-            __syncthreads();
-            // Warp w: M-block (w >> 1) of 32 rows, chunks (w & 1) * 8 .. +7; lane = chunk (low 3
-            // bits) + 8 * (8-row group inside the M-block). Each lane owns 8 rows x 8 columns.
-            const int chunk = (warp & 1) * 8 + (lane & 7);
-            const int rgq = lane >> 3;
-            const int mb = warp >> 1;
-            uint4 r[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) r[i] = tile[(mb * 32 + rgq * 8 + i) * 16 + chunk];
-            uint32_t m4[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t mm = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t word = (w == 0 ? r[i].x : w == 1 ? r[i].y : w == 2 ? r[i].z : r[i].w);
-                    mm = bf16x2_absmax(mm, word);
-                }
-                mm &= 0x7FFF7FFFu;
-                mm = max_u16x2(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 8));
-                mm = max_u16x2(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 16));
-                m4[w] = mm;
-            }
-            const int64_t kcol0 = rc.k0 + chunk * 8;
-            const int64_t mrow0 = rc.m0 + mb * 32;
-            const bool valid = rc.full || ((kcol0 < T.K) && (mrow0 < T.M));
-            uint8_t* qbase = T.q_col + kcol0 * T.M + mrow0 + rgq * 8;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int w = j >> 1, h = j & 1;
-                const uint32_t amax = h ? (m4[w] >> 16) : (m4[w] & 0xFFFFu);
-                const uint32_t s = scale_byte_from_amax(amax);
-                uint32_t e[8];       // (row i, column j) widened to fp32 bits
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t word = (w == 0 ? r[i].x : w == 1 ? r[i].y : w == 2 ? r[i].z : r[i].w);
-                    e[i] = h ? (word & 0xFFFF0000u) : (word << 16);
-                }
-                uint2 o;
-                if (s != 0xFFu) {
-                    const uint64_t inv2 = inv_scale2(s);
-                    o.x = enc_quad(e[0], e[1], e[2], e[3], inv2);
-                    o.y = enc_quad(e[4], e[5], e[6], e[7], inv2);
-                } else {
-                    o.x = 0x7F7F7F7Fu | ((e[0] >> 24) & 0x80u) | ((e[1] >> 16) & 0x8000u) |
-                          ((e[2] >> 8) & 0x800000u) | (e[3] & 0x80000000u);
-                    o.y = 0x7F7F7F7Fu | ((e[4] >> 24) & 0x80u) | ((e[5] >> 16) & 0x8000u) |
-                          ((e[6] >> 8) & 0x800000u) | (e[7] & 0x80000000u);
-                }
-                if (valid) *reinterpret_cast<uint2*>(qbase + j * T.M) = o;
-                if (rgq == 0) {
-                    const int kk = chunk * 8 + j;   // K-row inside the tile
-                    atom_col[(kk & 31) * 16 + (kk >> 5) * 4 + mb] = valid ? static_cast<uint8_t>(s) : 0;
-                }
-            }
-        }
-
-        __syncthreads();
-        // Scale output: one 512-byte block of the tensor-core layout per direction, or raw bytes.
-        if constexpr (ROW) {
-            if (a.swz) {
-                if (tid < 32)
-                    reinterpret_cast<uint4*>(T.s_row + (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512)[tid] =
-                        reinterpret_cast<const uint4*>(atom_row)[tid];
-            } else if (tid < kQTile) {
-                const int64_t m = rc.m0 + tid;
-                const int64_t nb = (kblocks - rc.kt * 4 < 4 ? kblocks - rc.kt * 4 : 4);
-                if (m < T.M)
-                    for (int b = 0; b < nb; ++b)
-                        T.s_row[m * kblocks + rc.kt * 4 + b] = atom_row[(tid & 31) * 16 + (tid >> 5) * 4 + b];
-            }
-        }
-        if constexpr (COL) {
-            const int64_t mblocks = T.M / 32;
-            const int u = tid - 128;
-            if (a.swz) {
-                if (u >= 0 && u < 32)
-                    reinterpret_cast<uint4*>(T.s_col + (static_cast<int64_t>(rc.kt) * T.tiles_m + rc.mt) * 512)[u] =
-                        reinterpret_cast<const uint4*>(atom_col)[u];
-            } else if (u >= 0) {
-                const int64_t k = rc.k0 + u;
-                const int64_t nb = (mblocks - rc.mt * 4 < 4 ? mblocks - rc.mt * 4 : 4);
-                if (k < T.K)
-                    for (int b = 0; b < nb; ++b)
-                        T.s_col[k * mblocks + rc.mt * 4 + b] = atom_col[(u & 31) * 16 + (u >> 5) * 4 + b];
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int it = 0; it < 8; ++it) cur[it] = nxt[it];
-        rc = rn;
-    }
 }
 
 // ---- rowwise-only kernel: one thread per 32-element block ----------------------------------
@@ -486,6 +306,202 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
             if (m < T.M)
                 for (int q = 0; q < nb; ++q)
                     T.s_row[m * kblocks + rc.kt * 4 + q] = atom[(tid & 31) * 16 + (tid >> 5) * 4 + q];
+        }
+        __syncthreads();
+        cur[0] = nxt[0];
+        cur[1] = nxt[1];
+        rc = rn;
+    }
+}
+
+// ---- rowwise + columnwise (or columnwise only) kernel --------------------------------------
+//
+// Same tile walk and block-per-thread rowwise pass as above. Each thread also stages its two
+// BF16 blocks in shared memory (128 rows x 256 bytes; 16-byte chunks XOR-swizzled so that both
+// these row-block writes and the column reads below are free of bank conflicts). Then thread t
+// quantizes tile columns 2 (t & 63) and 2 (t & 63) + 1 over the 32-row M-block t >> 6: each 32-bit
+// shared word holds one row's pair of those columns, so one pass of packed BF16 maxima gives both
+// columns' amax. Its 2 x 32 codes are two 32-byte pieces of the transposed copy ([K, M]).
+
+// Byte offset of 16-byte chunk c (0..15) of row r in the shared tile.
+__device__ __forceinline__ uint32_t qtile_chunk(int r, int c) {
+    return static_cast<uint32_t>(r * 256 + ((c ^ (((c >> 3) & 1) << 1) ^ (r & 1)) << 4));
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
+// The 32 BF16 of one column (the low or the high halves of w[0..31]) -> 32 E4M3 bytes, row i in
+// byte i of the result.
+__device__ __forceinline__ void encode_col32(const uint32_t (&w)[32], uint32_t s, bool hi, uint32_t (&o)[8]) {
+    if (s != 0xFFu) {
+        const uint64_t inv2 = inv_scale2(s);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint32_t e[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) e[i] = hi ? (w[4 * q + i] & 0xFFFF0000u) : (w[4 * q + i] << 16);
+            o[q] = enc_quad(e[0], e[1], e[2], e[3], inv2);
+        }
+    } else {
+        // NaN/Inf block: every element byte is sign | 0x7F.
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint32_t r = 0x7F7F7F7Fu;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t sign = hi ? (w[4 * q + i] >> 31) : ((w[4 * q + i] >> 15) & 1u);
+                r |= sign << (8 * i + 7);
+            }
+            o[q] = r;
+        }
+    }
+}
+
+template <bool ROW, int NT>
+__global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __grid_constant__ QuantArgs<NT> a) {
+    __shared__ __align__(128) uint8_t tile[kQTile * 256];
+    __shared__ __align__(16) uint8_t atom_row[512];
+    __shared__ __align__(16) uint8_t atom_col[512];
+    const int tid = threadIdx.x;
+    const uint32_t tile_s = smem_u32(tile);
+
+    const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
+    const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
+    const int64_t t_end = min(a.total_tiles, t_begin + per);
+    Block32 cur[2], nxt[2];
+    TileRef rc, rn;
+    if (t_begin < t_end) {
+        rc = decode_qtile(a, t_begin);
+        load_row_tile(a, rc, cur, tid);
+    }
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        if (t + 1 < t_end) {
+            rn = rc;
+            if (++rn.kt == a.t[rn.i].tiles_k) {
+                rn.kt = 0;
+                if (++rn.mt == a.t[rn.i].tiles_m) {
+                    rn.mt = 0;
+                    ++rn.i;
+                }
+            }
+            const QTensor& Tn = a.t[rn.i];
+            rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
+            rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
+            rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
+            load_row_tile(a, rn, nxt, tid);
+        }
+        const QTensor& T = a.t[rc.i];
+        const int kb = tid & 3;
+        const int64_t col = rc.k0 + kb * 32;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = h * 64 + (tid >> 2);           // row inside the tile
+            const Block32& b = cur[h];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                st_shared_v4(tile_s + qtile_chunk(r, kb * 4 + j), b.v[j].x, b.v[j].y, b.v[j].z, b.v[j].w);
+            if constexpr (ROW) {
+                const int64_t row = rc.m0 + r;
+                const bool valid = rc.full || (row < T.M && col < T.K);
+                uint32_t m = bf16x2_absmax(bf16x2_absmax(b.v[0].x, b.v[0].y), bf16x2_absmax(b.v[0].z, b.v[0].w));
+#pragma unroll
+                for (int j = 1; j < 4; ++j)
+                    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(b.v[j].x, b.v[j].y),
+                                                       bf16x2_absmax(b.v[j].z, b.v[j].w)));
+                m &= 0x7FFF7FFFu;
+                const uint32_t s = scale_byte_from_amax(max(m & 0xFFFFu, m >> 16));
+                uint4 o0, o1;
+                uint2 e;
+                e = encode_chunk(b.v[0], s);
+                o0.x = e.x; o0.y = e.y;
+                e = encode_chunk(b.v[1], s);
+                o0.z = e.x; o0.w = e.y;
+                e = encode_chunk(b.v[2], s);
+                o1.x = e.x; o1.y = e.y;
+                e = encode_chunk(b.v[3], s);
+                o1.z = e.x; o1.w = e.y;
+                if (valid) {
+                    uint8_t* q = T.q_row + row * T.K + col;
+                    if (T.vec32) {
+                        st_v8(q, o0, o1);
+                    } else {
+                        reinterpret_cast<uint4*>(q)[0] = o0;
+                        reinterpret_cast<uint4*>(q)[1] = o1;
+                    }
+                }
+                atom_row[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
+            }
+        }
+        __syncthreads();
+        {
+            const int cp = tid & 63;                     // column pair: tile columns 2 cp, 2 cp + 1
+            const int mb = tid >> 6;                     // 32-row M-block
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                w[i] = ld_shared_u32(tile_s + qtile_chunk(mb * 32 + i, cp >> 2) + (cp & 3) * 4);
+            uint32_t m = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m = bf16x2_absmax(m, w[i]);
+            m &= 0x7FFF7FFFu;
+            const int64_t kc = rc.k0 + 2 * cp;           // K-row of the transposed copy (low halves)
+            const int64_t mr = rc.m0 + 32 * mb;
+            const bool mok = rc.full || mr < T.M;        // M % 32 == 0: a block is all in or all out
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t s = scale_byte_from_amax(hh ? (m >> 16) : (m & 0xFFFFu));
+                const bool ok = mok && (rc.full || kc + hh < T.K);
+                uint32_t o[8];
+                encode_col32(w, s, hh != 0, o);
+                if (ok) {
+                    uint8_t* q = T.q_col + (kc + hh) * T.M + mr;
+                    const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
+                    const uint4 hi4 = make_uint4(o[4], o[5], o[6], o[7]);
+                    if (T.col_vec32) {
+                        st_v8(q, lo, hi4);
+                    } else {
+                        reinterpret_cast<uint4*>(q)[0] = lo;
+                        reinterpret_cast<uint4*>(q)[1] = hi4;
+                    }
+                }
+                const int kk = 2 * cp + hh;              // K-row inside the tile
+                atom_col[(kk & 31) * 16 + (kk >> 5) * 4 + mb] = ok ? static_cast<uint8_t>(s) : 0;
+            }
+        }
+        __syncthreads();
+        // Scale output: one 512-byte block of the tensor-core layout per direction, or raw bytes.
+        if constexpr (ROW) {
+            if (a.swz) {
+                if (tid < 32)
+                    reinterpret_cast<uint4*>(T.s_row + (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512)[tid] =
+                        reinterpret_cast<const uint4*>(atom_row)[tid];
+            } else if (tid < kQTile) {
+                const int64_t kblocks = T.K / 32;
+                const int64_t m_ = rc.m0 + tid;
+                const int64_t nb = (kblocks - rc.kt * 4 < 4 ? kblocks - rc.kt * 4 : 4);
+                if (m_ < T.M)
+                    for (int q = 0; q < nb; ++q)
+                        T.s_row[m_ * kblocks + rc.kt * 4 + q] = atom_row[(tid & 31) * 16 + (tid >> 5) * 4 + q];
+            }
+        }
+        {
+            const int64_t mblocks = T.M / 32;
+            const int u = tid - 128;
+            if (a.swz) {
+                if (u >= 0 && u < 32)
+                    reinterpret_cast<uint4*>(T.s_col + (static_cast<int64_t>(rc.kt) * T.tiles_m + rc.mt) * 512)[u] =
+                        reinterpret_cast<const uint4*>(atom_col)[u];
+            } else if (u >= 0) {
+                const int64_t k = rc.k0 + u;
+                const int64_t nb = (mblocks - rc.mt * 4 < 4 ? mblocks - rc.mt * 4 : 4);
+                if (k < T.K)
+                    for (int q = 0; q < nb; ++q)
+                        T.s_col[k * mblocks + rc.mt * 4 + q] = atom_col[(u & 31) * 16 + (u >> 5) * 4 + q];
+            }
         }
         __syncthreads();
         cur[0] = nxt[0];
