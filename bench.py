@@ -469,6 +469,120 @@ def run_secondary(device, peaks, reps=10):
     return out
 
 
+def run_library_gemm_peak(device, reps=10):
+    """Dense MXFP8 reference points at 8192^3, BF16 out: cuBLAS through torch `scaled_mm`
+    (BlockWise1x32 scales in the SWIZZLE_32_4_4 layout, fed with this library's bytes) and mx_gemm
+    on the same operands."""
+    import torch
+    import torch.nn.functional as F
+
+    from mxfp8_block_scaled_07_b200 import mx, synth
+
+    n = 8192
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    A = synth.normal_bf16((n, n), std=1.0, seed=51, device=device)
+    B = synth.normal_bf16((n, n), std=1.0, seed=52, device=device)
+    qa, sa, _, _ = mx.quantize(A, True, False)
+    qb, sb, _, _ = mx.quantize(B, True, False)
+    del A, B
+    C = torch.empty((n, n), dtype=torch.bfloat16, device=device)
+    flops = 2.0 * n * n * n
+    out = {"shape": "8192x8192x8192 bf16-out"}
+    ms = time_gpu(lambda: mx.gemm(qa, sa, qb, sb, out=C), reps, flush, stream)
+    out["mx_gemm_tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    try:
+        fa, fb = qa.view(torch.float8_e4m3fn), qb.view(torch.float8_e4m3fn).t()
+        ea, eb = sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu)
+        fn = lambda: F.scaled_mm(fa, fb, ea, F.ScalingType.BlockWise1x32, eb, F.ScalingType.BlockWise1x32,
+                                 swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                                 output_dtype=torch.bfloat16)
+        fn()
+        ms = time_gpu(fn, reps, flush, stream)
+        out["cublas_mxfp8_tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    except (RuntimeError, TypeError, NotImplementedError, AttributeError) as e:
+        out["cublas_mxfp8_tflops"] = None
+        out["cublas_note"] = f"torch scaled_mm MXFP8 unavailable: {type(e).__name__}"
+    torch.cuda.synchronize()
+    return out
+
+
+BREAKEVEN_TOKENS = (1312, 2592, 5216, 10304)   # 1.3k / 2.6k / 5.2k / 10.3k rounded to multiples of 32
+
+
+def run_breakeven(device, reps=20):
+    """Kernel-level fixed cost and per-token cost of one update micro-batch of a Qwen3-8B linear
+    (W 12288 x 4096, the TP-2 gate_up shard): BF16 (cuBLAS fprop, dgrad, wgrad) against MXFP8
+    (quantize X and dY row+col with the scale layout, then the three MXFP8 GEMMs), each micro-batch
+    one CUDA graph, L2 flushed before each replay. Fits t = delta + c * tokens per path (the pages'
+    stage cost model, Table 7) and reports the break-even tokens per micro-batch m* =
+    (delta_mxfp8 - delta_bf16) / (c_bf16 - c_mxfp8). The weight's own quantization happens once
+    per optimizer step, not per micro-batch, and is reported beside the fit."""
+    import torch
+
+    from mxfp8_block_scaled_07_b200 import mx, synth
+
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    O, H = 12288, 4096
+    W = synth.normal_bf16((O, H), std=0.02, seed=61, device=device)
+    qw = mx.quantize(W, True, True)
+    wq_ms = time_gpu(lambda: mx.quantize(W, True, True, out=qw), reps, flush, torch.cuda.current_stream())
+    rows = []
+    for T in BREAKEVEN_TOKENS:
+        X = synth.normal_bf16((T, H), std=1.0, seed=62, device=device)
+        dY = synth.normal_bf16((T, O), std=1e-3, seed=63, device=device)
+        Y = torch.empty((T, O), dtype=torch.bfloat16, device=device)
+        dX = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        dW = torch.empty((O, H), dtype=torch.bfloat16, device=device)
+        qx = mx.quantize(X, True, True)
+        qd = mx.quantize(dY, True, True)
+
+        def bf16_step():
+            torch.matmul(X, W.t(), out=Y)
+            torch.matmul(dY, W, out=dX)
+            torch.matmul(dY.t(), X, out=dW)
+
+        def mxfp8_step():
+            mx.quantize(X, True, True, out=qx)
+            mx.quantize(dY, True, True, out=qd)
+            mx.gemm(qx[0], qx[1], qw[0], qw[1], out=Y)
+            mx.gemm(qd[0], qd[1], qw[2], qw[3], out=dX)
+            mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW)
+
+        times = {}
+        for name, fn in (("bf16", bf16_step), ("mxfp8", mxfp8_step)):
+            with torch.cuda.stream(stream):
+                fn()                                  # warm-up outside capture
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            times[name] = time_gpu(g.replay, reps, flush, torch.cuda.current_stream())
+            del g
+        rows.append({"tokens": T, "bf16_ms": round(times["bf16"], 4), "mxfp8_ms": round(times["mxfp8"], 4)})
+        del X, dY, Y, dX, dW, qx, qd
+    torch.cuda.synchronize()
+
+    def fit(ys):
+        xs = [r["tokens"] for r in rows]
+        n = len(xs)
+        mx_, my = sum(xs) / n, sum(ys) / n
+        c = sum((x - mx_) * (y - my) for x, y in zip(xs, ys)) / sum((x - mx_) ** 2 for x in xs)
+        return my - c * mx_, c
+
+    d_b, c_b = fit([r["bf16_ms"] for r in rows])
+    d_m, c_m = fit([r["mxfp8_ms"] for r in rows])
+    dd, dc = d_m - d_b, c_b - c_m
+    return {"linear": "W 12288x4096 (fprop, dgrad, wgrad per micro-batch)", "points": rows,
+            "bf16": {"delta_ms": round(d_b, 4), "c_us_per_token": round(c_b * 1e3, 5)},
+            "mxfp8": {"delta_ms": round(d_m, 4), "c_us_per_token": round(c_m * 1e3, 5)},
+            "delta_delta_ms": round(dd, 4), "delta_c_us_per_token": round(dc * 1e3, 5),
+            "m_star_tokens": (round(dd / dc, 1) if dc > 0 else None),
+            "weight_quantize_row_col_ms_per_step": round(wq_ms, 4),
+            "timing": "one CUDA graph per micro-batch and path, median of 20 replays, L2 flushed before each"}
+
+
 CASES = ("quant-gate-up", "quant-dy-rowcol", "gemm-fwd-10300", "gemm-update-fprop", "gemm-moe-gate-up",
          "gemm-moe-down", "grid-equal-gate-up")
 
@@ -619,6 +733,8 @@ def main():
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_secondary:
         secondary = run_secondary(device, peaks)
+        secondary["dense_8192_reference"] = run_library_gemm_peak(device)
+        secondary["update_breakeven"] = run_breakeven(device)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         v, desc = oracle_sync_sample(12.0)
         cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
