@@ -200,7 +200,7 @@ class SyncWorkload:
         self.total_elems = 0
         self.compare_bytes = 0
         for layer, idx, r, c in sync_shapes():
-            W = synth.normal_bf16((r, c), std=0.02, seed=layer * 4 + idx + 144 * rank, device=device,
+            W = synth.normal_bf16((r, c), std=0.02, seed=rank_seed(layer, idx, rank), device=device,
                                   outlier_frac=1e-3, outlier_scale=50.0)
             # Sampler copy: dequantize the learner's grid to BF16 (exact here: every scale >= 2^-124)
             # and let the sampler re-derive elements and the tensor-core scale layout from it.
@@ -286,24 +286,35 @@ def barrier_sync(pg):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(pg, value: float) -> float:
+def max_over_ranks(pg, value: float, device="cuda") -> float:
+    """The slowest rank's time: the job's time (every rank does the same work, weak scaling)."""
     if pg is None:
         return value
     import torch
 
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(pg, value: int) -> int:
+def sum_over_ranks(pg, value: int, device="cuda") -> int:
     if pg is None:
         return value
     import torch
 
-    t = torch.tensor([value], dtype=torch.int64, device="cuda")
+    t = torch.tensor([value], dtype=torch.int64, device=device)
     pg.all_reduce(t)
     return int(t.item())
+
+
+def job_throughput_gbs(world: int, bytes_per_rank_step: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes all ranks processed in one step over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_max * 1e-3) / 1e9
+
+
+def rank_seed(layer: int, idx: int, rank: int) -> int:
+    """Seed of one weight tensor of one rank: every rank synchronizes its own 144 tensors."""
+    return layer * 4 + idx + 144 * rank
 
 
 def traffic_record():
@@ -706,7 +717,7 @@ def main():
     cmp_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
     ms = max_over_ranks(pg, ms_local)
     mismatches = sum_over_ranks(pg, int(wl.results[0].sum().item()))
-    value = world * wl.step_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput_gbs(world, wl.step_bytes, ms)
 
     quant_launch_ms = quant_ms          # one mx_quantize_multi launch per step
     quant_bytes_per_launch = wl.quant_bytes
