@@ -111,7 +111,10 @@ mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags
  * during the call) lists `groups` consecutive row counts summing to `rows`; every group is padded
  * to a multiple of 128 rows on its own and the groups' layouts are concatenated
  * (sum_g ceil(rows_g/128)*128 * ceil(kblocks/4)*4 bytes) -- the A-operand scale layout that
- * mx_grouped_gemm reads. Pad bytes are written 0.
+ * mx_grouped_gemm reads. Pad bytes are written 0. rows == 0 or kblocks == 0 is a no-op (pointers
+ * may then be NULL). Errors: MX_ERR_ARG (negative sizes or group rows, groups < 1 with a list,
+ * NULL pointers), MX_ERR_SHAPE (group rows not summing to rows), MX_ERR_ALIGN (s_swz not 16-byte
+ * aligned).
  */
 mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks,
                             const int64_t* group_rows_host, int64_t groups, uint8_t* s_swz,
@@ -125,8 +128,10 @@ mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks,
  *   sa_swz, sb_swz: scales of qa and qb in the tensor-core layout (as mx_quantize with
  *                   MX_SWIZZLE writes them) (device);
  *   c: device, row stride ld_c elements; rows >= M / columns >= N are never written.
- * Requirements: M, N >= 0, K > 0, K % 32 == 0, ld_c >= N, ld_c * sizeof(out) % 16 == 0, all
- * pointers 16-byte aligned, M, N, K < 2^31.
+ * Requirements: M, N >= 0, K > 0, K % 32 == 0, ld_c >= N, qa/sa_swz/qb/sb_swz 16-byte aligned,
+ * c aligned to its element size, M, N, K < 2^31. Rows of C that start 16-byte aligned (c and
+ * ld_c * sizeof(out) multiples of 16) are written with 16-byte stores, others element by element.
+ * M == 0 or N == 0 is a no-op (pointers may then be NULL).
  * Accuracy: |c - exact| <= 1e-5 * sum_k |a_k b_k| (+ 2^-8 |exact| for BF16 output).
  */
 mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz,

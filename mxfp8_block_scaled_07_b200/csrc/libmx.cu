@@ -406,9 +406,8 @@ mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags
 
 mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, const int64_t* group_rows_host,
                             int64_t groups, uint8_t* s_swz, mx_stream stream) {
-    if (!s || !s_swz || rows < 0 || kblocks < 0) return MX_ERR_ARG;
+    if (rows < 0 || kblocks < 0) return MX_ERR_ARG;
     if (group_rows_host && groups < 1) return MX_ERR_ARG;
-    if (!aligned16(s_swz)) return MX_ERR_ALIGN;
     if (group_rows_host) {
         int64_t total = 0;
         for (int64_t g = 0; g < groups; ++g) {
@@ -417,7 +416,9 @@ mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, con
         }
         if (total != rows) return MX_ERR_SHAPE;
     }
-    if (rows == 0 || kblocks == 0) return MX_OK;
+    if (rows == 0 || kblocks == 0) return MX_OK;   // empty: pointers may be NULL
+    if (!s || !s_swz) return MX_ERR_ARG;
+    if (!aligned16(s_swz)) return MX_ERR_ALIGN;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
 

@@ -97,6 +97,8 @@ def test_swizzle_and_grid_equal_argument_errors(L):
     assert s(FAKE, 8, 4, ctypes.cast(rows, ctypes.c_void_p), 2, FAKE, None) == -2   # groups do not sum to rows
     neg = (ctypes.c_int64 * 2)(-1, 8)
     assert s(FAKE, 7, 4, ctypes.cast(neg, ctypes.c_void_p), 2, FAKE, None) == -1
+    assert s(None, 0, 4, None, 0, None, None) == 0        # empty: a no-op, NULL pointers allowed
+    assert s(None, 4, 0, None, 0, None, None) == 0
     e = L.mx_grid_equal
     assert e(FAKE, FAKE, 16, None, FAKE, None) == -1
     assert e(FAKE, FAKE, -1, FAKE, FAKE, None) == -1
