@@ -92,6 +92,7 @@ struct GemmArgs {
     int out_bf16;
     int vec_store;      // output rows 16-byte aligned: full 16-byte chunks use 16-byte stores
     int G;
+    int n_fast;         // dense: consecutive tiles step along N (B re-read from L2, A streamed once)
     int n_rowtiles;     // ceil(N / 128): scale row-tiles of one B operand
     const int32_t* row_offsets;
     uint32_t* err;
@@ -123,7 +124,9 @@ template <bool GROUPED>
 __device__ __forceinline__ Tile decode_tile1(int t, const GemmArgs& a, const int32_t* off, const int32_t* pm) {
     Tile T;
     if constexpr (!GROUPED) {
-        const int mt = t % a.tiles_m, nt = t / a.tiles_m;
+        // Tile walk: the smaller operand stays resident in L2 while the larger one streams once.
+        const int mt = a.n_fast ? t / a.tiles_n : t % a.tiles_m;
+        const int nt = a.n_fast ? t % a.tiles_n : t / a.tiles_m;
         T.a_row0 = mt * kBM;
         T.rows_valid = min(kBM, a.M - T.a_row0);
         T.n0 = nt * kBN;
@@ -153,7 +156,9 @@ __device__ __forceinline__ Tile decode_tile_pair(int t, int rank, const GemmArgs
     Tile T;
     int sf_last_in_b;
     if constexpr (!GROUPED) {
-        const int mt = t % a.tiles_m, nt = t / a.tiles_m;
+        // Tile walk: the smaller operand stays resident in L2 while the larger one streams once.
+        const int mt = a.n_fast ? t / a.tiles_n : t % a.tiles_m;
+        const int nt = a.n_fast ? t % a.tiles_n : t / a.tiles_m;
         T.a_row0 = mt * 2 * kBM + rank * kBM;
         T.rows_valid = max(0, min(kBM, a.M - T.a_row0));
         T.n0 = nt * kBN;

@@ -512,6 +512,7 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     a.out_bf16 = out_dtype == MX_OUT_BF16;
     a.vec_store = vector_store_ok(c, ld_c, out_dtype);
     a.G = 1;
+    a.n_fast = M > N;      // A is the larger operand: walk N fastest so B (the smaller) stays in L2
     a.n_rowtiles = static_cast<int>(ceil_div(N, 128));
     a.row_offsets = nullptr;
     a.err = d->status;
