@@ -652,8 +652,8 @@ def run_breakeven(device, reps=20):
             "timing": "one CUDA graph per micro-batch and path, median of 20 replays, L2 flushed before each"}
 
 
-CASES = ("quant-gate-up", "quant-dy-rowcol", "gemm-fwd-10300", "gemm-update-fprop", "gemm-moe-gate-up",
-         "gemm-moe-down", "grid-equal-gate-up")
+CASES = ("quant-gate-up", "quant-dy-rowcol", "gemm-fwd-10300", "gemm-update-fprop", "gemm-update-dgrad",
+         "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up")
 
 
 def run_case(name: str, reps: int):
@@ -689,6 +689,12 @@ def run_case(name: str, reps: int):
         offs = torch.tensor(synth.group_offsets(counts), dtype=torch.int32, device=dev)
         C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
         fn = lambda: mx.grouped_gemm(qa, sa, qb.reshape(G, N, K), sb, offs, out=C)
+    elif name == "gemm-update-dgrad":
+        _, W, dY = synth.update_inputs(device=dev)
+        qd, sd, _, _ = mx.quantize(dY, True, False)
+        _, _, qwc, swc = mx.quantize(W, False, True)
+        C = torch.empty((dY.shape[0], W.shape[1]), dtype=torch.bfloat16, device=dev)
+        fn = lambda: mx.gemm(qd, sd, qwc, swc, out=C)
     else:
         if name == "gemm-fwd-10300":
             A = synth.fwd_activations(10300, device=dev)

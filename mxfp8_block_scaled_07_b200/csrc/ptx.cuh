@@ -132,8 +132,10 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
                  : "memory");
     return v;
 }
+// Streaming store (evict-first in L2): GEMM output is written once and not read back here, so it
+// should not displace the operand tiles other CTAs are about to read from L2.
 __device__ __forceinline__ void st_global_v4(void* p, const uint4& v) {
-    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+    asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 
