@@ -65,6 +65,8 @@ def _load():
     lib.oracle_gemm.restype = None
     lib.oracle_grouped_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     lib.oracle_grouped_gemm.restype = None
+    lib.oracle_swiglu_quantize.argtypes = [P, I64, I64, P, P, P]
+    lib.oracle_swiglu_quantize.restype = ctypes.c_int
     lib.oracle_grid_equal.argtypes = [P, P, I64, P, P]
     lib.oracle_grid_equal.restype = None
     _lib = lib
@@ -184,6 +186,20 @@ def grouped_gemm(qa, sa, qb, sb, row_offsets):
     a = np.empty((qa.shape[0], N), np.float64)
     _load().oracle_grouped_gemm(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), _ptr(off), G, N, K, _ptr(c), _ptr(a))
     return c, a
+
+
+def swiglu_quantize(gu):
+    """gu: fp64 [rows, 2n] (gate features, then up features) -> (h fp64 [rows, n], q uint8
+    [rows, n], s uint8 [rows, n/32]): h = silu(gate) * up, then the rowwise MXFP8 rule on h."""
+    gu = np.ascontiguousarray(gu, np.float64)
+    rows, n2 = gu.shape
+    n = n2 // 2
+    h = np.empty((rows, n), np.float64)
+    q = np.empty((rows, n), np.uint8)
+    s = np.empty((rows, n // 32), np.uint8)
+    if _load().oracle_swiglu_quantize(_ptr(gu), rows, n, _ptr(h), _ptr(q), _ptr(s)) != 0:
+        raise ValueError("n must be a multiple of 32")
+    return h, q, s
 
 
 def grid_equal(a: np.ndarray, b: np.ndarray):

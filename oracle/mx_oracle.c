@@ -222,6 +222,40 @@ void oracle_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb
     }
 }
 
+/* ---- SwiGLU activation + MXFP8 rule (fp64) -------------------------------------------------- */
+
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+
+int oracle_swiglu_quantize(const double* gu, int64_t rows, int64_t n, double* h, uint8_t* q, uint8_t* s) {
+    if (n % 32 != 0) return -1;
+    double v[32];
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < n / 32; ++b) {
+            double amax = 0.0;
+            int special = 0;
+            for (int i = 0; i < 32; ++i) {
+                const int64_t f = b * 32 + i;
+                v[i] = silu(gu[r * 2 * n + f]) * gu[r * 2 * n + n + f];
+                if (h) h[r * n + f] = v[i];
+                if (isnan(v[i]) || isinf(v[i])) special = 1;
+                else if (fabs(v[i]) > amax) amax = fabs(v[i]);
+            }
+            uint8_t* qb = q + r * n + b * 32;
+            if (special) {
+                /* same NaN/Inf policy as the BF16 quantizer */
+                for (int i = 0; i < 32; ++i) qb[i] = (uint8_t)((signbit(v[i]) ? 0x80 : 0) | 0x7F);
+                s[r * (n / 32) + b] = 0xFF;
+                continue;
+            }
+            const uint8_t sc = oracle_e8m0_scale(amax);
+            const int e = (int)sc - 127;
+            for (int i = 0; i < 32; ++i) qb[i] = oracle_e4m3_encode(ldexp(v[i], -e));
+            s[r * (n / 32) + b] = sc;
+        }
+    }
+    return 0;
+}
+
 /* ---- byte comparison ---------------------------------------------------------------------- */
 
 void oracle_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes,

@@ -74,6 +74,15 @@ void oracle_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb
                          const uint8_t* sb, const int64_t* row_offsets, int64_t groups,
                          int64_t N, int64_t K, double* c, double* abs_sum);
 
+/* The MoE expert MLP's activation between its two GEMMs, then the MXFP8 rule on the result
+ * (Table 2: Qwen3-30B-A3B experts; the down projection consumes this activation quantized):
+ *   h[r, f] = silu(gu[r, f]) * gu[r, n + f],  silu(x) = x / (1 + exp(-x)),  f < n,
+ * from the gate_up product gu [rows, 2n] (gate features first, then up features), all in fp64.
+ * Each row of h is then quantized in 32-blocks exactly as a rowwise BF16 tensor would be
+ * (same scale rule, same rounding), from the fp64 values. Writes h (fp64, may be NULL),
+ * q [rows, n] and raw scales s [rows, n / 32]. Returns -1 if n % 32 != 0. */
+int oracle_swiglu_quantize(const double* gu, int64_t rows, int64_t n, double* h, uint8_t* q, uint8_t* s);
+
 /* Byte comparison: number of positions i with a[i] != b[i] and the first such i (-1 if none). */
 void oracle_grid_equal(const uint8_t* a, const uint8_t* b, int64_t nbytes,
                        uint64_t* mismatches, int64_t* first_index);

@@ -367,3 +367,50 @@ def test_grid_equal_matches_numpy():
     b[idx] ^= g.integers(1, 256, idx.size, dtype=np.uint8)
     assert oracle.grid_equal(a, b) == (37, int(idx[0]))
     assert oracle.grid_equal(a[:0], b[:0]) == (0, -1)
+
+
+# ---- SwiGLU + MXFP8 rule on the expert activation -----------------------------------------
+
+
+def test_swiglu_quantize_reduces_to_the_bf16_quantizer_for_saturated_gates():
+    # For gate = 2^k with k >= 6, sigmoid(gate) rounds to exactly 1 in fp64, so h = gate * up is
+    # exact and BF16-representable (up BF16, gate a power of two): the result must equal the
+    # (independently pinned) BF16 rowwise quantizer applied to that BF16 tensor.
+    g = np.random.default_rng(21)
+    rows, n = 6, 96
+    up = synth.normal_bf16((rows, n), std=3.0, seed=22, outlier_frac=0.05, outlier_scale=40.0)
+    gate = np.ldexp(1.0, g.integers(6, 40, (rows, n)))
+    gu = np.concatenate([gate, up.double().numpy()], axis=1)
+    h, q, s = oracle.swiglu_quantize(gu)
+    hb = torch.from_numpy(gate * up.double().numpy()).to(torch.bfloat16)
+    assert np.array_equal(hb.double().numpy(), h)          # h is exactly gate * up
+    q_ref, s_ref = oracle.quantize_rowwise(hb)
+    assert np.array_equal(q, q_ref) and np.array_equal(s, s_ref)
+
+
+def test_swiglu_quantize_special_cases():
+    n = 32
+    # up = 0: h = +-0 (sign of silu(gate)); all-zero block -> scale 0, codes 0x00 / 0x80.
+    gate = np.linspace(-5.0, 5.0, n)
+    gu = np.concatenate([gate, np.zeros(n)])[None, :]
+    h, q, s = oracle.swiglu_quantize(gu)
+    assert np.all(h == 0.0) and s[0, 0] == 0
+    assert np.array_equal(q[0], np.where(gate < 0, 0x80, 0x00).astype(np.uint8))
+    # gate = ln 3: sigmoid = 3/4, so h = 0.75 ln(3) up.
+    up = np.linspace(-2.0, 2.0, n)
+    gu = np.concatenate([np.full(n, math.log(3.0)), up])[None, :]
+    h, _, _ = oracle.swiglu_quantize(gu)
+    assert np.allclose(h[0], 0.75 * math.log(3.0) * up, rtol=4e-16, atol=0.0)
+    with pytest.raises(ValueError):
+        oracle.swiglu_quantize(np.zeros((1, 2 * 48)))
+
+
+def test_swiglu_odd_part_is_gate_times_up():
+    # silu(x) - silu(-x) = x, so h(g, u) - h(-g, u) = g u: a check of the sign and of which half
+    # is the gate.
+    g = np.random.default_rng(23)
+    gate = g.normal(0.0, 3.0, (4, 64))
+    up = g.normal(0.0, 1.0, (4, 64))
+    h1, _, _ = oracle.swiglu_quantize(np.concatenate([gate, up], axis=1))
+    h2, _, _ = oracle.swiglu_quantize(np.concatenate([-gate, up], axis=1))
+    assert np.allclose(h1 - h2, gate * up, rtol=1e-13, atol=1e-14)
