@@ -533,6 +533,40 @@ def run_secondary(device, peaks, reps=10):
         add_gemm(f"{name} grouped {rows}x{N}x{K} (128 experts)", 2.0 * rows * N * K,
                  lambda: mx.grouped_gemm(qa, sa, qb, sb, offs, out=C))
         del qa, sa_raw, sa, qb, sb, C
+    # gate_up with SwiGLU and the down GEMM's MXFP8 quantization fused into the epilogue, against the
+    # unfused chain (gate_up GEMM to BF16, SwiGLU in torch, quantize + grouped scale layout).
+    G, N2, K = W1.shape
+    n = N2 // 2
+    qa, sa_raw, _, _ = mx.quantize(Xp, True, False, swizzle=False)
+    sa = mx.swizzle_scales(sa_raw, counts)
+    W1i = W1.view(G, 2, n // 128, 128, K).permute(0, 2, 1, 3, 4).reshape(G * N2, K).contiguous()
+    qbi, sbi, _, _ = mx.quantize(W1i, True, False)
+    qbi = qbi.reshape(G, N2, K)
+    hq = mx.grouped_gemm_swiglu_quant(qa, sa, qbi, sbi, offs, counts)
+    fused_ms = time_gpu(lambda: mx.grouped_gemm_swiglu_quant(qa, sa, qbi, sbi, offs, counts, out=hq), reps, flush,
+                        stream)
+    qb, sb, _, _ = mx.quantize(W1.reshape(G * N2, K), True, False)
+    qb = qb.reshape(G, N2, K)
+    C = torch.empty((rows, N2), dtype=torch.bfloat16, device=device)
+    hbuf = mx.quantize(torch.empty((rows, n), dtype=torch.bfloat16, device=device), True, False, swizzle=False)
+    hs = torch.empty(mx.grouped_swizzled_scale_bytes(counts, n // 32), dtype=torch.uint8, device=device)
+
+    def unfused():
+        mx.grouped_gemm(qa, sa, qb, sb, offs, out=C)
+        h = (torch.nn.functional.silu(C[:, :n].float()) * C[:, n:].float()).to(torch.bfloat16)
+        mx.quantize(h, True, False, swizzle=False, out=hbuf)
+        mx.swizzle_scales(hbuf[1], counts, out=hs)
+
+    unfused()
+    unfused_ms = time_gpu(unfused, reps, flush, stream)
+    flops = 2.0 * rows * N2 * K
+    out["moe_gate_up_swiglu_quant"] = {
+        "workload": f"moe gate_up {rows}x{N2}x{K} + SwiGLU + MXFP8 quantize of h (128 experts)",
+        "fused_ms": round(fused_ms, 4), "fused_tflops": round(flops / (fused_ms * 1e-3) / 1e12, 1),
+        "unfused_ms": round(unfused_ms, 4),
+        "unfused": "mx_grouped_gemm (BF16 out) + torch SwiGLU + mx_quantize + mx_swizzle_scales",
+        "speedup": round(unfused_ms / fused_ms, 3)}
+    del qa, sa_raw, sa, W1i, qbi, sbi, hq, qb, sb, C, hbuf, hs
     del Xp, Hh, W1, W2
     torch.cuda.synchronize()
     return out

@@ -159,6 +159,35 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
                           mx_out_dtype out_dtype, mx_stream stream);
 
 /*
+ * The expert MLP's first GEMM with its activation and the down GEMM's quantization fused into the
+ * epilogue (Table 2: Qwen3-30B-A3B experts, whose down projection consumes this activation in
+ * MXFP8). For every group g and row r in [off[g], off[g+1]), with gu = A[r, :] . B_g^T:
+ *   h[r, f] = silu(gate[r, f]) * up[r, f],  silu(x) = x / (1 + exp(-x)),  f < n_inter,
+ * computed in fp32 from the fp32 accumulator, then quantized rowwise like mx_quantize does a
+ * BF16 tensor (32-blocks along f; E8M0 scale from the block's fp32 amax, e = floor(log2 amax) - 8
+ * clamped to [-127, 127]; codes RNE(h * 2^-e) saturated to +-448; 0xFF scale and sign|0x7F codes
+ * for a block holding NaN or Inf). No BF16 gate_up or h is written.
+ *   qa, sa_swz, row_offsets_dev, G, total_rows, K: as mx_grouped_gemm;
+ *   qb[G, 2 n_inter, K], sb_swz: the experts' gate and up weights with their rows interleaved per
+ *           128: rows [256 t, 256 t + 128) of expert g are gate rows [128 t, 128 t + 128), rows
+ *           [256 t + 128, 256 t + 256) the up rows of the same features; scales as mx_grouped_gemm;
+ *   h_q[total_rows, n_inter]: E4M3 codes (device, packed);
+ *   h_s_swz: h's scales in the grouped tensor-core layout (each group padded to 128 rows; the size
+ *           mx_swizzle_scales gives for [total_rows, n_inter / 32] with the groups' row counts),
+ *           pad bytes written 0 -- the A-operand scales mx_grouped_gemm reads for the down GEMM.
+ * Requirements: n_inter % 128 == 0, h_q and h_s_swz 16-byte aligned, and those of
+ * mx_grouped_gemm. Always runs the CTA-pair kernel.
+ * Accuracy: h differs from the exact value by the GEMM's error propagated through SwiGLU plus
+ * fp32 rounding of exp, the division and the products, so a code can differ from the exactly
+ * rounded one where h lies that close to a rounding boundary, and a scale where the block's amax
+ * lies that close to a power of two.
+ */
+mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
+                                       const uint8_t* sb_swz, const int32_t* row_offsets_dev, int64_t G,
+                                       int64_t total_rows, int64_t n_inter, int64_t K, uint8_t* h_q,
+                                       uint8_t* h_s_swz, mx_stream stream);
+
+/*
  * Selects the kernel behind later mx_gemm / mx_grouped_gemm calls (process-wide): 0 (default) the
  * CTA-pair kernel (256 x 256 tiles computed by two SMs with tcgen05.mma.cta_group::2), 1 the
  * single-CTA kernel (128 x 256 tiles). Both meet the accuracy bound above; results may differ in

@@ -32,6 +32,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "quantize.cuh"    // the E4M3 encoding helpers, shared with the fused SwiGLU epilogue
 
 namespace mx {
 
@@ -97,6 +98,12 @@ struct GemmArgs {
     const int32_t* row_offsets;
     uint32_t* err;
     uint64_t timeout_ns;
+    // Fused SwiGLU + MXFP8 epilogue (grouped gate_up GEMM): the quantized activation [M, n_inter],
+    // its scales in the grouped tensor-core layout (hs_ctiles = n_inter / 128 blocks per 128 rows).
+    uint8_t* hq;
+    uint8_t* hs;
+    int n_inter;
+    int hs_ctiles;
 };
 
 // What one CTA does for one tile.
@@ -320,6 +327,98 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
     }
 }
 
+// Fused epilogue of the expert gate_up GEMM: SwiGLU, then the MXFP8 rule, straight into the down
+// GEMM's operand. The caller interleaves the weight rows per 128, so tile columns [0, 128) hold the
+// gate features f0 .. f0 + 127 and [128, 256) the up features of the same f0 (f0 = 128 * tile
+// column index). Each thread (one row) computes h = silu(gate) * up in fp32 from the fp32
+// accumulator, 32 features at a time; the block's E8M0 scale comes from the fp32 amax (OCP rule:
+// e = floor(log2 amax) - 8, clamped at -127, i.e. byte = biased exponent - 8, at least 0; 0xFF when
+// the block holds NaN or Inf), the codes from one satfinite E4M3 rounding of h * 2^-e (exact
+// power-of-two scaling). 32 code bytes go to hq[row, f0 + 32 b .. ], the 4 scale bytes of the row as
+// one word into the grouped tensor-core layout (the CTA's 128 rows are one 128-row scale tile,
+// T.sfa_tile, as for the A operand). Rows past the expert's end write zero scale bytes (the
+// layout's pad rows) and no codes.
+__device__ __forceinline__ void epilogue_swiglu_tile(const GemmArgs& a, const Tile& T, uint32_t tmem_base,
+                                                     bool acc1, uint32_t ovl_free_addr, uint32_t acc_empty_addr,
+                                                     int q, int lane) {
+    const int row_local = q * 32 + lane;
+    const bool row_ok = row_local < T.rows_valid;
+    const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
+
+    uint32_t ov[16];                     // tile columns 240..255 of accumulator 0, 0..15 of accumulator 1
+    tc_ld_32x32b_x16(lanes + kOvlCol, ov);
+    tc_wait_ld_regs(ov);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
+
+    auto load32 = [&](int c, uint32_t(&p)[32]) {
+        if (acc1 && c == 0) {
+            tc_ld_32x32b_x16(tq + 16u, *reinterpret_cast<uint32_t(*)[16]>(&p[16]));
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = ov[i];
+        } else if (!acc1 && c == 7) {
+            tc_ld_32x32b_x16(tq + 224u, *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[16 + i] = ov[i];
+        } else {
+            tc_ld_32x32b_x32(tq + 32u * c, p);
+        }
+    };
+    const int nt = T.n0 / kBN;
+    uint8_t* hrow = a.hq + (static_cast<int64_t>(T.a_row0) + row_local) * a.n_inter + nt * 128;
+    uint32_t sbytes = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t gw[32], uw[32];
+        load32(b, gw);                   // gate features f0 + 32 b ..
+        load32(4 + b, uw);               // up features of the same f0 + 32 b ..
+        tc_wait_ld_regs(gw, uw);
+        if (b == 3) {                    // every TMEM load of the tile has landed
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_addr);
+        }
+        float amax = 0.0f;
+        bool special = false;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(gw[i]);
+            const float h = g / (1.0f + expf(-g)) * __uint_as_float(uw[i]);
+            special |= !(fabsf(h) <= 3.402823466e38f);   // NaN or Inf
+            amax = fmaxf(amax, fabsf(h));
+            gw[i] = __float_as_uint(h);
+        }
+        const uint32_t E = __float_as_uint(amax) >> 23;
+        const uint32_t sc = special ? 0xFFu : (E > 8u ? E - 8u : 0u);
+        uint32_t o[8];
+        if (!special) {
+            const uint64_t inv2 = inv_scale2(sc);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[k] = enc_quad(gw[4 * k], gw[4 * k + 1], gw[4 * k + 2], gw[4 * k + 3], inv2);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                uint32_t r = 0x7F7F7F7Fu;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) r |= (gw[4 * k + i] >> 31) << (8 * i + 7);
+                o[k] = r;
+            }
+        }
+        if (row_ok) {
+            uint4* d = reinterpret_cast<uint4*>(hrow + 32 * b);
+            d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        sbytes |= (row_ok ? sc : 0u) << (8 * b);
+    }
+    if (T.rows_valid > 0) {
+        const int64_t blk = static_cast<int64_t>(T.sfa_tile) * a.hs_ctiles + nt;
+        *reinterpret_cast<uint32_t*>(a.hs + blk * 512 + lane * 16 + q * 4) = sbytes;
+    }
+}
+
 // Loads the group row offsets into shared memory, checks them and builds the prefix sums of
 // row tiles per group (tile_rows = 128: pm128; also 256: pm256 when given). Returns the tile count
 // (0 and an error bit when the offsets are invalid). Executed by the whole CTA.
@@ -520,7 +619,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ---------------------------------------------------------------------------------------------
 constexpr uint32_t kPairStageBytes = kBM * kBK + (kBN / 2) * kBK + kSfaBytes + kSfbBytes;   // per CTA
 
-template <bool GROUPED>
+// EPI 0: C written as fp32 / BF16; EPI 1 (grouped only): the fused SwiGLU + MXFP8 epilogue.
+template <bool GROUPED, int EPI = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
@@ -681,7 +781,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait(&tmem_full[g], full_phase, abort, a.err, a.timeout_ns)) break;
             full_phase ^= 1u;
             tc_fence_after();
-            epilogue_tile<GROUPED>(a, T, tmem_base, g != 0, stage, ovl_addr, empty_addr, q, lane);
+            if constexpr (EPI == 0)
+                epilogue_tile<GROUPED>(a, T, tmem_base, g != 0, stage, ovl_addr, empty_addr, q, lane);
+            else
+                epilogue_swiglu_tile(a, T, tmem_base, g != 0, ovl_addr, empty_addr, q, lane);
         }
     }
 

@@ -123,6 +123,8 @@ const DeviceInfo* device_info() {
             cudaFuncSetAttribute(mx_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmPairSmemDense) != cudaSuccess ||
             cudaFuncSetAttribute(mx_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmPairSmemGrouped) != cudaSuccess ||
+            cudaFuncSetAttribute(mx_gemm_pair_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmPairSmemGrouped) != cudaSuccess)
             return nullptr;
         d.pair_clusters[0] = max_pair_clusters(mx_gemm_pair_kernel<false>, kGemmPairSmemDense, d.sms);
@@ -210,7 +212,7 @@ bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t blocks) {
 }
 
 // Launches the CTA-pair GEMM with a cluster dimension of 2.
-template <bool GROUPED>
+template <bool GROUPED, int EPI = 0>
 mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
                       const CUtensorMap& tsb, const GemmArgs& a, mx_stream stream) {
     cudaLaunchConfig_t cfg = {};
@@ -225,7 +227,7 @@ mx_status launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<GROUPED>, ta, tb, tsa, tsb, a) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<GROUPED, EPI>, ta, tb, tsa, tsb, a) != cudaSuccess) {
         cudaGetLastError();
         return MX_ERR_CUDA;
     }
@@ -586,6 +588,52 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, d->sms));
     mx_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemGrouped, stream>>>(ta, tb, a);
     return launched();
+}
+
+mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
+                                       const uint8_t* sb_swz, const int32_t* row_offsets_dev, int64_t G,
+                                       int64_t total_rows, int64_t n_inter, int64_t K, uint8_t* h_q,
+                                       uint8_t* h_s_swz, mx_stream stream) {
+    if (!row_offsets_dev || G < 1 || n_inter <= 0) return MX_ERR_ARG;
+    if (G > kMaxGroups || n_inter % 128 != 0) return MX_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(row_offsets_dev) & 3u) return MX_ERR_ALIGN;
+    const int64_t N = 2 * n_inter;
+    bool empty = false;
+    // Operand and shape checks of the GEMM (its C argument stands in for h_q here; h_q and h_s_swz
+    // get their own 16-byte alignment check below).
+    if (mx_status st = gemm_checks(qa, sa_swz, qb, sb_swz, total_rows, N, K, h_q, N, MX_OUT_BF16, &empty))
+        return st;
+    if (G * N >= (int64_t(1) << 31)) return MX_ERR_SHAPE;
+    if (empty) return MX_OK;
+    if (!h_s_swz) return MX_ERR_ARG;
+    if (!aligned16(h_q) || !aligned16(h_s_swz)) return MX_ERR_ALIGN;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    GemmArgs a{};
+    a.sfa = sa_swz;
+    a.sfb = sb_swz;
+    a.M = static_cast<int>(total_rows);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.nkb = static_cast<int>(ceil_div(K, kBK));
+    a.tiles_n = static_cast<int>(N / kBN);
+    a.G = static_cast<int>(G);
+    a.n_rowtiles = static_cast<int>(N / 128);
+    a.row_offsets = row_offsets_dev;
+    a.err = d->status;
+    a.timeout_ns = g_timeout_ns.load();
+    a.hq = h_q;
+    a.hs = h_s_swz;
+    a.n_inter = static_cast<int>(n_inter);
+    a.hs_ctiles = static_cast<int>(n_inter / 128);
+    const int64_t max_tiles = (ceil_div(total_rows, 2 * kBM) + G) * a.tiles_n;
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kBN / 2) ||
+        !make_tmap_sf(&tsa, sa_swz, (ceil_div(total_rows, 128) + G) * a.nkb) ||
+        !make_tmap_sf(&tsb, sb_swz, G * a.n_rowtiles * a.nkb))
+        return MX_ERR_CUDA;
+    const int pairs = static_cast<int>(std::min<int64_t>(max_tiles, d->pair_clusters[1]));
+    return launch_pair<true, 1>(pairs, ta, tb, tsa, tsb, a, stream);
 }
 
 void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }

@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.mx_swizzle_scales.restype = I32
     L.mx_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, I32, P]
     L.mx_gemm.restype = I32
+    L.mx_grouped_gemm_swiglu_quant.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_swiglu_quant.restype = I32
     L.mx_grouped_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, I32, P]
     L.mx_grouped_gemm.restype = I32
     L.mx_grid_equal.argtypes = [P, P, I64, P, P, P]
@@ -225,6 +227,25 @@ def grouped_gemm(qa, sa_swz, qb, sb_swz, row_offsets, out_dtype=torch.bfloat16, 
                                out.stride(0), _out_code(out.dtype), ctypes.c_void_p(_stream(qa.device)))
     _check(st, "mx_grouped_gemm")
     return out
+
+
+def grouped_gemm_swiglu_quant(qa, sa_swz, qb, sb_swz, row_offsets, group_rows, out=None):
+    """mx_grouped_gemm_swiglu_quant. qb: [G, 2 n, K] with gate/up rows interleaved per 128;
+    group_rows: rows per expert (host), for the size of h's grouped scale layout. Returns
+    (h_q uint8 [total, n], h_s uint8 grouped tensor-core layout of [total, n / 32])."""
+    total, K = qa.shape
+    G, N2, K2 = qb.shape
+    assert K2 == K and N2 % 2 == 0 and row_offsets.dtype == torch.int32 and row_offsets.numel() == G + 1
+    n = N2 // 2
+    if out is None:
+        u8 = dict(dtype=torch.uint8, device=qa.device)
+        out = (torch.empty((total, n), **u8),
+               torch.empty(grouped_swizzled_scale_bytes([int(r) for r in group_rows], n // 32), **u8))
+    hq, hs = out
+    st = lib().mx_grouped_gemm_swiglu_quant(_p(qa), _p(sa_swz), _p(qb), _p(sb_swz), _p(row_offsets), G, total, n,
+                                            K, _p(hq), _p(hs), ctypes.c_void_p(_stream(qa.device)))
+    _check(st, "mx_grouped_gemm_swiglu_quant")
+    return hq, hs
 
 
 def grid_equal(a: torch.Tensor, b: torch.Tensor, out=None):

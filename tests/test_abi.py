@@ -87,6 +87,14 @@ def test_gemm_argument_errors(L):
     assert gg(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 8, 32, FAKE, 8, 0, None) == -1
     assert gg(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 8, 32, FAKE, 8, 0, None) == -1
     assert gg(FAKE, FAKE, FAKE, FAKE, FAKE, 1025, 64, 8, 32, FAKE, 8, 0, None) == -2
+    sq = L.mx_grouped_gemm_swiglu_quant     # (qa, sa, qb, sb, off, G, rows, n_inter, K, h_q, h_s, stream)
+    assert sq(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 128, 32, FAKE, FAKE, None) == -1
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 128, 32, FAKE, FAKE, None) == -1
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 96, 32, FAKE, FAKE, None) == -2      # n_inter % 128
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 128, 48, FAKE, FAKE, None) == -2     # K % 32
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 128, 32, FAKE_ODD, FAKE, None) == -3  # h_q alignment
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 128, 32, FAKE, None, None) == -1     # no h_s
+    assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 128, 32, None, None, None) == 0       # empty: no-op
 
 
 def test_swizzle_and_grid_equal_argument_errors(L):
