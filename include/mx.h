@@ -178,7 +178,8 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
  * Requirements: n_inter % 128 == 0, h_q and h_s_swz 16-byte aligned, and those of
  * mx_grouped_gemm. Always runs the CTA-pair kernel.
  * Accuracy: h differs from the exact value by the GEMM's error propagated through SwiGLU plus
- * fp32 rounding of exp, the division and the products, so a code can differ from the exactly
+ * the error of CUDA's __expf and __fdividef (a few ulps, growing with |gate|) and the fp32
+ * products, so a code can differ from the exactly
  * rounded one where h lies that close to a rounding boundary, and a scale where the block's amax
  * lies that close to a power of two.
  */

@@ -331,7 +331,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
 // GEMM's operand. The caller interleaves the weight rows per 128, so tile columns [0, 128) hold the
 // gate features f0 .. f0 + 127 and [128, 256) the up features of the same f0 (f0 = 128 * tile
 // column index). Each thread (one row) computes h = silu(gate) * up in fp32 from the fp32
-// accumulator, 32 features at a time; the block's E8M0 scale comes from the fp32 amax (OCP rule:
+// accumulator, 32 features at a time, with CUDA's fast __expf and __fdividef (their error, a few
+// ulps growing with |gate|, is part of the stated accuracy); the block's E8M0 scale comes from the fp32 amax (OCP rule:
 // e = floor(log2 amax) - 8, clamped at -127, i.e. byte = biased exponent - 8, at least 0; 0xFF when
 // the block holds NaN or Inf), the codes from one satfinite E4M3 rounding of h * 2^-e (exact
 // power-of-two scaling). 32 code bytes go to hq[row, f0 + 32 b .. ], the 4 scale bytes of the row as
@@ -385,7 +386,7 @@ __device__ __forceinline__ void epilogue_swiglu_tile(const GemmArgs& a, const Ti
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float g = __uint_as_float(gw[i]);
-            const float h = g / (1.0f + expf(-g)) * __uint_as_float(uw[i]);
+            const float h = g * __fdividef(1.0f, 1.0f + __expf(-g)) * __uint_as_float(uw[i]);
             special |= !(fabsf(h) <= 3.402823466e38f);   // NaN or Inf
             amax = fmaxf(amax, fabsf(h));
             gw[i] = __float_as_uint(h);

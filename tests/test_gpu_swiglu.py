@@ -35,9 +35,11 @@ def check_against_oracle(gu, abs_sum, q_k, s_k):
     g, u = gu[:, :n], gu[:, n:]
     sig = 1.0 / (1.0 + np.exp(-g))
     silu = g * sig
-    # |dh| <= |dh/dg| dg + |dh/du| du + fp32 roundings of exp, divide and two products.
+    # |dh| <= |dh/dg| dg + |dh/du| du + fp32 roundings: __expf (relative error about
+    # (2 + 1.2 |g|) ulps), __fdividef (2 ulps) and the two products.
     tol_g, tol_u = 1e-5 * abs_sum[:, :n] + 1e-30, 1e-5 * abs_sum[:, n:] + 1e-30
-    d = np.abs(u * (sig + g * sig * (1.0 - sig))) * tol_g + np.abs(silu) * tol_u + 8 * 2.0 ** -24 * np.abs(h_ref)
+    d = (np.abs(u * (sig + g * sig * (1.0 - sig))) * tol_g + np.abs(silu) * tol_u
+         + (8.0 + 2.0 * np.abs(g)) * 2.0 ** -23 * np.abs(h_ref))
     hb, db = h_ref.reshape(rows, n // 32, 32), d.reshape(rows, n // 32, 32)
     amax = np.abs(hb).max(axis=2)
     dmax = db.max(axis=2)
