@@ -15,6 +15,9 @@
 //     both. Per SM this halves B traffic and the scale-copy work per FLOP against one CTA alone.
 //   mx_gemm_kernel: one CTA computes a 128 x 256 tile with cta_group::1 MMAs.
 //
+// The pair kernel's EPI = 1 instantiation (grouped only) replaces the C store with the MoE expert
+// activation and the down projection's MXFP8 quantization (epilogue_swiglu_tile).
+//
 // Roles (320 threads): warp 0 TMA producer (A/B tiles with the 128-byte swizzle, scale blocks);
 // warp 1 TMEM owner and MMA issuer; warps 2-9 epilogue in two groups of four (warp w reads TMEM
 // lanes 32 * (w % 4); group (w - 2) / 4 drains one accumulator, i.e. every other tile).
@@ -22,7 +25,8 @@
 // ([496, 508)): the epilogue drains the shared columns first, so the next tile's MMAs start while
 // the rest of the previous tile is still being read out. tcgen05 operations issued by one thread
 // execute in order, so a scale copy never overtakes the MMAs that read the slot's previous contents.
-// The epilogue writes through per-warp swizzled staging and coalesced 16-byte stores.
+// The epilogue writes through per-warp swizzled staging and coalesced 16-byte stores. Tiles walk M
+// first, or N first when A is the larger operand, so the smaller operand stays in L2.
 //
 // Every mbarrier wait is bounded (globaltimer deadline); on expiry the kernel records an error bit,
 // stops all roles, drains its in-flight copies and MMAs, frees TMEM and returns. No load uses
