@@ -213,6 +213,27 @@ def oracle_sync_sample_parallel(max_procs: int = 16):
     return gbs, procs, desc
 
 
+def oracle_gemm_sample(rows: int = 2):
+    """The oracle GEMM (plain fp64 C, one thread) on a row sample of the dense forward config
+    (10300 x 24576 x 4096): `rows` full output rows. Returns (FLOP/s, description with the
+    full-size time extrapolated from it)."""
+    import oracle
+    from mxfp8_block_scaled_07_b200 import synth
+
+    oracle.build()
+    X = synth.fwd_activations(rows)                   # the first rows of the forward activations
+    W = synth.sync_weight(0, 2)                        # gate_up 24576 x 4096
+    qx, sx = oracle.quantize_rowwise(X)
+    qw, sw = oracle.quantize_rowwise(W)
+    t0 = time.perf_counter()
+    oracle.gemm(qx, sx, qw, sw)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * W.shape[0] * W.shape[1]
+    full = 2.0 * 10300 * W.shape[0] * W.shape[1] / (flops / dt)
+    return flops / dt, (f"oracle GEMM (plain C, fp64, 1 thread): {rows} full rows of fwd 10300x24576x4096 in "
+                        f"{dt:.1f} s; full size extrapolated: {full / 3600:.1f} h")
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -847,8 +868,10 @@ def main():
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         v1, desc1 = oracle_sync_sample(12.0)
         vp, procs, descp = oracle_sync_sample_parallel()
+        gf, gdesc = oracle_gemm_sample()
         cpu = {"value": round(vp, 4), "unit": UNIT, "cores": procs, "kind": "oracle", "sample": descp,
-               "single_thread": {"value": round(v1, 4), "cores": 1, "sample": desc1}}
+               "single_thread": {"value": round(v1, 4), "cores": 1, "sample": desc1},
+               "gemm": {"value": round(gf / 1e9, 3), "unit": "GFLOP/s", "cores": 1, "sample": gdesc}}
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
