@@ -460,6 +460,17 @@ def run_e2e(wl, args, device):
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 2), "steps": steps, "grid_equal": ok}
 
 
+def aggregate_e2e(pg, local: dict, world: int, bytes_per_rank_step: int, device="cuda") -> dict:
+    """Whole-job end-to-end figures from each rank's run_e2e: the slowest rank's step time, all
+    ranks' bytes, and grid equality on every rank."""
+    ms = max_over_ranks(pg, local["ms_per_step"], device=device)
+    bad = sum_over_ranks(pg, 0 if local["grid_equal"] else 1, device=device)
+    return {"value": round(job_throughput_gbs(world, bytes_per_rank_step, ms), 2), "unit": UNIT,
+            "h2d_bytes_per_step": world * local["h2d_bytes_per_step"],
+            "d2h_bytes_per_step": world * local["d2h_bytes_per_step"],
+            "ms_per_step": round(ms, 2), "steps": local["steps"], "grid_equal": bad == 0}
+
+
 def flush_l2(buf):
     buf.add_(1)
 
@@ -856,12 +867,13 @@ def main():
     secondary = None
     e2e = None
     cpu = None
-    if rank == 0:
-        if not args.no_e2e:
-            e2e = run_e2e(wl, args, device)
+    if not args.no_e2e:                  # every rank: the whole job's end-to-end step
+        e2e = aggregate_e2e(pg, run_e2e(wl, args, device), world, wl.step_bytes)
     del wl
     torch.cuda.empty_cache()
-    if rank == 0 and not args.no_secondary:
+    # Kernel characterization lines (one GPU's kernels) only in single-GPU runs: the other ranks
+    # of a multi-GPU run would otherwise wait for them inside a collective.
+    if rank == 0 and not args.no_secondary and world == 1:
         secondary = run_secondary(device, peaks)
         secondary["dense_8192_reference"] = run_library_gemm_peak(device)
         secondary["update_breakeven"] = run_breakeven(device)

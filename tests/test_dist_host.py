@@ -35,7 +35,10 @@ def _rank_main(rank, world, port, out_dir):
         dist.barrier()
         ms = bench.max_over_ranks(dist, 1.0 + rank * 0.5, device="cpu")
         mism = bench.sum_over_ranks(dist, 3 * rank + 1, device="cpu")
-        res = {"ms": ms, "mismatches": mism,
+        e2e = bench.aggregate_e2e(dist, {"ms_per_step": 100.0 + 10 * rank, "grid_equal": rank == 0,
+                                         "h2d_bytes_per_step": 7, "d2h_bytes_per_step": 3, "steps": 3},
+                                  world, 10 ** 9, device="cpu")
+        res = {"ms": ms, "mismatches": mism, "e2e": e2e,
                "value": bench.job_throughput_gbs(world, 10 ** 9, ms),
                "seeds": [bench.rank_seed(layer, idx, rank) for layer in range(36) for idx in range(4)]}
         # The reference arm under torchrun: ranks other than 0 exit at once with status 0.
@@ -62,5 +65,10 @@ def test_two_gloo_ranks_aggregate_like_the_bench(tmp_path):
         assert x["mismatches"] == 1 + 4                     # summed over ranks
         assert x["value"] == pytest.approx(2 * 1e9 / 1.5e-3 / 1e9)
     assert r[1]["reference_rc"] == 0
+    for x in r:
+        e = x["e2e"]
+        assert e["ms_per_step"] == 110.0 and e["grid_equal"] is False     # rank 1 reported a mismatch
+        assert e["value"] == pytest.approx(2 * 1e9 / 0.110 / 1e9, rel=1e-3)
+        assert e["h2d_bytes_per_step"] == 14 and e["d2h_bytes_per_step"] == 6
     # Every rank synchronizes its own tensors: no seed is shared between ranks.
     assert len(set(r[0]["seeds"]) | set(r[1]["seeds"])) == 2 * 144
