@@ -65,6 +65,8 @@ def _load():
     lib.oracle_gemm.restype = None
     lib.oracle_grouped_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     lib.oracle_grouped_gemm.restype = None
+    lib.oracle_quantize_block128.argtypes = [P, I64, I64, I64, ctypes.c_int, P, P]
+    lib.oracle_quantize_block128.restype = None
     lib.oracle_swiglu_quantize.argtypes = [P, I64, I64, P, P, P]
     lib.oracle_swiglu_quantize.restype = ctypes.c_int
     lib.oracle_grid_equal.argtypes = [P, P, I64, P, P]
@@ -186,6 +188,17 @@ def grouped_gemm(qa, sa, qb, sb, row_offsets):
     a = np.empty((qa.shape[0], N), np.float64)
     _load().oracle_grouped_gemm(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), _ptr(off), G, N, K, _ptr(c), _ptr(a))
     return c, a
+
+
+def quantize_block128(x, pow2: bool):
+    """x: BF16 [M, K] -> (q uint8 [M, K], scales float32 [ceil(M/128), ceil(K/128)]): FP8 blockwise
+    with FP32 scales (pow2=False) or power-of-two scales (pow2=True)."""
+    xb = _bits(x)
+    M, K = xb.shape
+    q = np.empty((M, K), np.uint8)
+    s = np.empty(((M + 127) // 128, (K + 127) // 128), np.float32)
+    _load().oracle_quantize_block128(_ptr(xb), M, K, K, 1 if pow2 else 0, _ptr(q), _ptr(s))
+    return q, s
 
 
 def swiglu_quantize(gu):

@@ -222,6 +222,51 @@ void oracle_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb
     }
 }
 
+/* ---- FP8 blockwise, 128 x 128 blocks, FP32 or power-of-two scales -------------------------- */
+
+void oracle_quantize_block128(const uint16_t* x, int64_t M, int64_t K, int64_t ld, int pow2, uint8_t* q,
+                              float* scales) {
+    const int64_t bm = (M + 127) / 128, bk = (K + 127) / 128;
+    for (int64_t i = 0; i < bm; ++i) {
+        for (int64_t j = 0; j < bk; ++j) {
+            const int64_t r1 = (i + 1) * 128 < M ? (i + 1) * 128 : M;
+            const int64_t c1 = (j + 1) * 128 < K ? (j + 1) * 128 : K;
+            double amax = 0.0;
+            int special = 0;
+            for (int64_t r = i * 128; r < r1; ++r)
+                for (int64_t c = j * 128; c < c1; ++c) {
+                    const double v = bf16_to_double(x[r * ld + c]);
+                    if (isnan(v) || isinf(v)) special = 1;
+                    else if (fabs(v) > amax) amax = fabs(v);
+                }
+            float s;
+            if (special) {
+                s = NAN;
+            } else if (amax == 0.0) {
+                s = 1.0f;
+            } else {
+                s = (float)amax / 448.0f;                  /* IEEE single division */
+                if (pow2) {
+                    const int e = ilogbf(s);
+                    const float p = ldexpf(1.0f, e);
+                    s = (p == s) ? p : ldexpf(1.0f, e + 1);
+                }
+            }
+            scales[i * bk + j] = s;
+            for (int64_t r = i * 128; r < r1; ++r)
+                for (int64_t c = j * 128; c < c1; ++c) {
+                    const float v = (float)bf16_to_double(x[r * ld + c]);
+                    if (special) {
+                        q[r * K + c] = (uint8_t)((signbit(v) ? 0x80 : 0) | 0x7F);
+                    } else {
+                        const float t = v / s;                /* IEEE single division */
+                        q[r * K + c] = oracle_e4m3_encode((double)t);
+                    }
+                }
+        }
+    }
+}
+
 /* ---- SwiGLU activation + MXFP8 rule (fp64) -------------------------------------------------- */
 
 static double silu(double x) { return x / (1.0 + exp(-x)); }

@@ -74,6 +74,17 @@ void oracle_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb
                          const uint8_t* sb, const int64_t* row_offsets, int64_t groups,
                          int64_t N, int64_t K, double* c, double* abs_sum);
 
+/* FP8 blockwise quantization with one scale per 128 x 128 block of a BF16 weight x[M, K] (the
+ * "FP8 blockwise" recipe of Table 1, whose learner and sampler differ in their scales on SM100:
+ * power-of-two against FP32; Table 10 F6). amax = max |x| over the block. FP32 scales
+ * (pow2 == 0): s = fl32(amax / 448); codes RNE_E4M3(fl32(x / s)) saturated to +-448, both
+ * divisions in IEEE single precision. Power-of-two scales (pow2 != 0): s = the smallest power of
+ * two >= fl32(amax / 448); codes RNE_E4M3(x / s). An all-zero block takes s = 1; a block holding
+ * NaN or Inf takes s = NaN and codes sign | 0x7F. q[M, K]; scales[ceil(M/128), ceil(K/128)] fp32.
+ * Edge blocks cover what exists. */
+void oracle_quantize_block128(const uint16_t* x, int64_t M, int64_t K, int64_t ld, int pow2, uint8_t* q,
+                              float* scales);
+
 /* The MoE expert MLP's activation between its two GEMMs, then the MXFP8 rule on the result
  * (Table 2: Qwen3-30B-A3B experts; the down projection consumes this activation quantized):
  *   h[r, f] = silu(gu[r, f]) * gu[r, n + f],  silu(x) = x / (1 + exp(-x)),  f < n,

@@ -414,3 +414,61 @@ def test_swiglu_odd_part_is_gate_times_up():
     h1, _, _ = oracle.swiglu_quantize(np.concatenate([gate, up], axis=1))
     h2, _, _ = oracle.swiglu_quantize(np.concatenate([-gate, up], axis=1))
     assert np.allclose(h1 - h2, gate * up, rtol=1e-13, atol=1e-14)
+
+
+# ---- FP8 blockwise, 128 x 128 blocks, FP32 or power-of-two scales ----------------------------
+
+
+def test_block128_reduces_to_mxfp8_when_the_scale_is_a_power_of_two():
+    # Every 32-block holds one element of magnitude 448 * 2^k (the 128 x 128 block's amax), so
+    # amax / 448 = 2^k exactly: both scale modes give s = 2^k, and the MXFP8 rule gives every
+    # 32-block the same scale 2^k (floor(log2(448 * 2^k)) - 8 = k). Codes must then equal the
+    # (independently pinned) MXFP8 rowwise quantizer's.
+    g = np.random.default_rng(31)
+    for k in (-9, 0, 5):
+        x = torch.from_numpy(g.normal(0.0, 2.0 ** k * 40.0, (128, 256)))
+        x = torch.clamp(x, -448 * 2.0 ** k, 448 * 2.0 ** k)
+        x[:, ::32] = 448 * 2.0 ** k * torch.sign(torch.from_numpy(g.normal(size=(128, 8))))
+        xb = x.to(torch.bfloat16)
+        q_mx, s_mx = oracle.quantize_rowwise(xb)
+        assert np.all(s_mx == 127 + k)
+        for pow2 in (False, True):
+            q, s = oracle.quantize_block128(xb, pow2)
+            assert np.all(s == np.float32(2.0 ** k))
+            assert np.array_equal(q, q_mx)
+
+
+def test_block128_scale_properties():
+    g = np.random.default_rng(32)
+    x = torch.from_numpy(g.normal(0.0, 0.02, (256, 384)) * np.exp(g.normal(0.0, 2.0, (256, 384)))).to(torch.bfloat16)
+    xd = x.double().numpy()
+    q32, s32 = oracle.quantize_block128(x, False)
+    q2, s2 = oracle.quantize_block128(x, True)
+    dec = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    for i in range(2):
+        for j in range(3):
+            blk = xd[128 * i:128 * (i + 1), 128 * j:128 * (j + 1)]
+            amax = np.abs(blk).max()
+            a = np.unravel_index(np.abs(blk).argmax(), blk.shape)
+            # FP32 scale: the amax element lands on +-448.
+            assert abs(dec[q32[128 * i + a[0], 128 * j + a[1]]]) == 448.0
+            assert s32[i, j] == np.float32(np.float32(amax) / np.float32(448.0))
+            # Power-of-two scale: the power of two that brackets amax / 448 from above.
+            e = math.log2(float(s2[i, j]))
+            assert e == int(e) and s2[i, j] >= s32[i, j] and s2[i, j] < 2 * s32[i, j]
+            assert 224.0 <= abs(dec[q2[128 * i + a[0], 128 * j + a[1]]]) <= 448.0
+    # The two grids differ on generic weights: the gap the FP8-blockwise pairing carries.
+    assert np.mean(q32 != q2) > 0.3
+
+
+def test_block128_special_blocks_and_edges():
+    x = torch.zeros((130, 160), dtype=torch.bfloat16)
+    x[0, 0] = float("nan")                       # block (0, 0): NaN policy
+    x[129, 150] = -3.0                           # edge block (1, 1): 2 x 32 elements
+    for pow2 in (False, True):
+        q, s = oracle.quantize_block128(x, pow2)
+        assert s.shape == (2, 2) and np.isnan(s[0, 0])
+        assert np.all(q[:128, :128] == 0x7F) and s[0, 1] == 1.0 and s[1, 0] == 1.0
+        assert np.all(q[:128, 128:] == 0) and np.all(q[128:, :128] == 0)
+        q_edge, s_edge = oracle.quantize_block128(x[128:, 128:].contiguous(), pow2)
+        assert s[1, 1] == s_edge[0, 0] and np.array_equal(q[128:, 128:], q_edge)
