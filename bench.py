@@ -565,6 +565,33 @@ def run_secondary(device, peaks, reps=10):
         add_gemm(f"{name} grouped {rows}x{N}x{K} (128 experts)", 2.0 * rows * N * K,
                  lambda: mx.grouped_gemm(qa, sa, qb, sb, offs, out=C))
         del qa, sa_raw, sa, qb, sb, C
+    # FP8-blockwise grids of one weight (128 x 128 blocks): FP32 scales (the sampler's) against
+    # power-of-two scales (the learner's on SM100), beside the MXFP8 grid both sides share here.
+    W = synth.sync_weight(0, 2, device=device)
+    Mw, Kw = W.shape
+    g32 = mx.quantize_block128(W, False)
+    g2 = mx.quantize_block128(W, True)
+    ms32 = time_gpu(lambda: mx.quantize_block128(W, False, out=g32), reps, flush, stream)
+    ms2 = time_gpu(lambda: mx.quantize_block128(W, True, out=g2), reps, flush, stream)
+    cnt, _ = mx.grid_equal(g32[0], g2[0])
+
+    def deq_block(q, sc):
+        return q.view(torch.float8_e4m3fn).float() * sc.repeat_interleave(128, 0)[:Mw].repeat_interleave(128, 1)[:, :Kw]
+
+    qm, sm, _, _ = mx.quantize(W, True, False, swizzle=False)
+    dm = qm.view(torch.float8_e4m3fn).float() * torch.exp2(sm.float() - 127.0).repeat_interleave(32, dim=1)
+    d32, d2, ref = deq_block(*g32), deq_block(*g2), W.float()
+    bw_bytes = Mw * Kw * 3 + 4 * (Mw // 128) * (Kw // 128)
+    out["fp8_blockwise_gap"] = {
+        "workload": f"qwen3-8b gate_up {Mw}x{Kw}: FP8 blockwise (128x128) with FP32 vs power-of-two scales",
+        "byte_mismatch_frac": round(int(cnt.item()) / (Mw * Kw), 4),
+        "rel_diff_between_grids": round(float((d32 - d2).norm() / d32.norm()), 5),
+        "rel_err_fp32_scales": round(float((d32 - ref).norm() / ref.norm()), 5),
+        "rel_err_pow2_scales": round(float((d2 - ref).norm() / ref.norm()), 5),
+        "rel_err_mxfp8": round(float((dm - ref).norm() / ref.norm()), 5),
+        "quantize_gbs": {"fp32_scales": round(bw_bytes / (ms32 * 1e-3) / 1e9, 1),
+                         "pow2_scales": round(bw_bytes / (ms2 * 1e-3) / 1e9, 1)}}
+    del W, g32, g2, qm, sm, dm, d32, d2, ref
     # gate_up with SwiGLU and the down GEMM's MXFP8 quantization fused into the epilogue, against the
     # unfused chain (gate_up GEMM to BF16, SwiGLU in torch, quantize + grouped scale layout).
     G, N2, K = W1.shape

@@ -189,6 +189,23 @@ mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz,
                                        uint8_t* h_s_swz, mx_stream stream);
 
 /*
+ * FP8 blockwise quantization with one scale per 128 x 128 block (Table 1: the FP8-blockwise
+ * learner/sampler pairing, whose scales differ on SM100 -- power-of-two for the learner, FP32 for
+ * the sampler; Table 10 F6), to measure that pairing's grid gap beside the shared MXFP8 grid.
+ * amax = max |x| over the block. pow2_scales == 0: s = fl32(amax / 448) and codes
+ * RNE_E4M3(fl32(x / s)) saturated to +-448 (IEEE single divisions). pow2_scales != 0: s = the
+ * smallest power of two >= fl32(amax / 448) and codes RNE_E4M3(x / s). An all-zero block takes
+ * s = 1; a block holding NaN or Inf takes s = NaN and codes sign|0x7F.
+ *   x: BF16 [M, K] (device), row stride ld_x elements; q: [M, K] E4M3 codes (device, packed);
+ *   scales: fp32 [ceil(M/128), ceil(K/128)] row-major (device).
+ * Requirements: K % 32 == 0, ld_x >= K, ld_x % 8 == 0, x and q 16-byte aligned, scales 4-byte
+ * aligned. M == 0 or K == 0 is a no-op (pointers may then be NULL).
+ * Errors: MX_ERR_ARG, MX_ERR_SHAPE, MX_ERR_ALIGN as stated; MX_ERR_CUDA on a failed launch.
+ */
+mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x, int pow2_scales, uint8_t* q,
+                               float* scales, mx_stream stream);
+
+/*
  * Selects the kernel behind later mx_gemm / mx_grouped_gemm calls (process-wide): 0 (default) the
  * CTA-pair kernel (256 x 256 tiles computed by two SMs with tcgen05.mma.cta_group::2), 1 the
  * single-CTA kernel (128 x 256 tiles). Both meet the accuracy bound above; results may differ in

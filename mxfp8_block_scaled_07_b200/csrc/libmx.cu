@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/mx.h"
+#include "blockwise.cuh"
 #include "gemm.cuh"
 #include "grid_equal.cuh"
 #include "ptx.cuh"
@@ -634,6 +635,35 @@ mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz,
         return MX_ERR_CUDA;
     const int pairs = static_cast<int>(std::min<int64_t>(max_tiles, d->pair_clusters[1]));
     return launch_pair<true, 1>(pairs, ta, tb, tsa, tsb, a, stream);
+}
+
+mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x, int pow2_scales, uint8_t* q,
+                               float* scales, mx_stream stream) {
+    if (M < 0 || K < 0) return MX_ERR_ARG;
+    if (K % 32 != 0) return MX_ERR_SHAPE;
+    if (M == 0 || K == 0) return MX_OK;                // empty: pointers may be NULL
+    if (!x || !q || !scales) return MX_ERR_ARG;
+    if (ld_x < K) return MX_ERR_SHAPE;
+    if (!aligned16(x) || ld_x % 8 != 0 || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return MX_ERR_ALIGN;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    Block128Args a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.q = q;
+    a.scales = scales;
+    a.M = M;
+    a.K = K;
+    a.ldx = ld_x;
+    a.tiles_m = static_cast<int>(ceil_div(M, kQTile));
+    a.tiles_k = static_cast<int>(ceil_div(K, kQTile));
+    a.pow2 = pow2_scales != 0;
+    a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (ld_x % 16 == 0) &&
+              (reinterpret_cast<uintptr_t>(q) % 32 == 0);
+    const int64_t tiles = int64_t(a.tiles_m) * a.tiles_k;
+    const int64_t grid = std::min<int64_t>(tiles, int64_t(d->sms) * 4);
+    quantize_block128_kernel<<<grid, kQThreads, 0, stream>>>(a);
+    return launched();
 }
 
 void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }

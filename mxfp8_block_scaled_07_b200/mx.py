@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.mx_swizzle_scales.restype = I32
     L.mx_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, I32, P]
     L.mx_gemm.restype = I32
+    L.mx_quantize_block128.argtypes = [P, I64, I64, I64, I32, P, P, P]
+    L.mx_quantize_block128.restype = I32
     L.mx_grouped_gemm_swiglu_quant.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_swiglu_quant.restype = I32
     L.mx_grouped_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, I32, P]
@@ -246,6 +248,22 @@ def grouped_gemm_swiglu_quant(qa, sa_swz, qb, sb_swz, row_offsets, group_rows, o
                                             K, _p(hq), _p(hs), ctypes.c_void_p(_stream(qa.device)))
     _check(st, "mx_grouped_gemm_swiglu_quant")
     return hq, hs
+
+
+def quantize_block128(x: torch.Tensor, pow2_scales: bool, out=None):
+    """mx_quantize_block128 on a 2-D BF16 CUDA tensor: FP8 blockwise codes with one FP32
+    (pow2_scales=False) or power-of-two (pow2_scales=True) scale per 128 x 128 block.
+    Returns (q uint8 [M, K], scales float32 [ceil(M/128), ceil(K/128)])."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    if out is None:
+        out = (torch.empty((M, K), dtype=torch.uint8, device=x.device),
+               torch.empty(((M + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=x.device))
+    q, sc = out
+    st = lib().mx_quantize_block128(_p(x), M, K, x.stride(0), 1 if pow2_scales else 0, _p(q), _p(sc),
+                                    ctypes.c_void_p(_stream(x.device)))
+    _check(st, "mx_quantize_block128")
+    return q, sc
 
 
 def grid_equal(a: torch.Tensor, b: torch.Tensor, out=None):

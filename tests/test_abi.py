@@ -95,6 +95,14 @@ def test_gemm_argument_errors(L):
     assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 128, 32, FAKE_ODD, FAKE, None) == -3  # h_q alignment
     assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 128, 32, FAKE, None, None) == -1     # no h_s
     assert sq(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 128, 32, None, None, None) == 0       # empty: no-op
+    bq = L.mx_quantize_block128              # (x, M, K, ld_x, pow2, q, scales, stream)
+    assert bq(FAKE, -1, 64, 64, 0, FAKE, FAKE, None) == -1
+    assert bq(FAKE, 64, 48, 64, 0, FAKE, FAKE, None) == -2                      # K % 32
+    assert bq(FAKE, 64, 64, 32, 0, FAKE, FAKE, None) == -2                      # ld_x < K
+    assert bq(FAKE_ODD, 64, 64, 64, 0, FAKE, FAKE, None) == -3                  # x alignment
+    assert bq(FAKE, 64, 64, 64, 1, FAKE, ctypes.c_void_p(0x10002), None) == -3  # scales alignment
+    assert bq(None, 64, 64, 64, 0, FAKE, FAKE, None) == -1
+    assert bq(None, 0, 64, 64, 0, None, None, None) == 0                        # empty: no-op
 
 
 def test_swizzle_and_grid_equal_argument_errors(L):
