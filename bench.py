@@ -491,6 +491,15 @@ def time_gpu(fn, reps, flush_buf, stream):
     return statistics.median(times)
 
 
+def guarded(fn):
+    """A characterization line that fails reports its error in the JSON line instead of taking
+    the headline measurement down with it."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
 def run_secondary(device, peaks, reps=10):
     """GEMM TFLOP/s on the dense forward, update and MoE configs; quantize GB/s on activations."""
     import torch
@@ -901,9 +910,9 @@ def main():
     # Kernel characterization lines (one GPU's kernels) only in single-GPU runs: the other ranks
     # of a multi-GPU run would otherwise wait for them inside a collective.
     if rank == 0 and not args.no_secondary and world == 1:
-        secondary = run_secondary(device, peaks)
-        secondary["dense_8192_reference"] = run_library_gemm_peak(device)
-        secondary["update_breakeven"] = run_breakeven(device)
+        secondary = guarded(lambda: run_secondary(device, peaks))
+        secondary["dense_8192_reference"] = guarded(lambda: run_library_gemm_peak(device))
+        secondary["update_breakeven"] = guarded(lambda: run_breakeven(device))
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         v1, desc1 = oracle_sync_sample(12.0)
         vp, procs, descp = oracle_sync_sample_parallel()
