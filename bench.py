@@ -417,47 +417,89 @@ def traffic_record():
     return rec
 
 
+E2E_CHUNK = 16          # tensors per pipeline chunk of the end-to-end step
+
+
 def run_e2e(wl, args, device):
     """Same metric through the C ABI with host buffers: per step, every BF16 weight goes
     host(pinned) -> device, is quantized and compared on the device, and the learner grid (elements
-    + swizzled scales) and the comparison results come back to pinned host memory."""
+    + swizzled scales) and the comparison results come back to pinned host memory. The 144 tensors
+    move in chunks of E2E_CHUNK on three streams (copies in, kernels, copies out), so chunk c's
+    kernels overlap chunk c+1's upload and chunk c-1's download; each chunk is one
+    mx_quantize_multi and one mx_grid_equal_multi call. A chunk's device buffers are reused by the
+    next step only after its kernels (for the upload) and its download (for the kernels) are done."""
     import torch
 
-    from mxfp8_block_scaled_07_b200 import mx
-
-    stream = torch.cuda.current_stream()
+    s_in, s_k, s_out = (torch.cuda.Stream(device) for _ in range(3))
     host_w = [W.cpu().pin_memory() for (W, _, _, _, _) in wl.items]
     host_q = [torch.empty(q.shape, dtype=torch.uint8).pin_memory() for (_, q, _, _, _) in wl.items]
     host_s = [torch.empty(s.shape, dtype=torch.uint8).pin_memory() for (_, _, s, _, _) in wl.items]
     host_r = torch.empty(wl.results.shape, dtype=torch.int64).pin_memory()
     h2d = sum(t.numel() * 2 for t in host_w)
     d2h = sum(t.numel() for t in host_q) + sum(t.numel() for t in host_s) + host_r.numel() * 8
-    sp = stream.cuda_stream
+    n = len(wl.items)
+    chunks = [(i0, min(n, i0 + E2E_CHUNK)) for i0 in range(0, n, E2E_CHUNK)]
+    from mxfp8_block_scaled_07_b200 import mx
+
+    qarrs = [mx.quant_tensor_array([it[0] for it in wl.items[i0:i1]], [(q, s, None, None) for (_, q, s, _, _) in
+                                                                      wl.items[i0:i1]]) for i0, i1 in chunks]
+    parrs = []
+    for i0, i1 in chunks:
+        pairs = []
+        for (_, q, s, qs, ss) in wl.items[i0:i1]:
+            pairs += [(q, qs), (s, ss)]
+        parrs.append(mx.compare_pair_array(pairs))
+    done_k = [None] * len(chunks)       # kernels of chunk c finished (its inputs may be overwritten)
+    done_out = [None] * len(chunks)     # download of chunk c finished (its outputs may be overwritten)
 
     def one_step():
-        for i, (W, q, s, qs, ss) in enumerate(wl.items):
-            W.copy_(host_w[i], non_blocking=True)
-        wl.quantize_all(ctypes.c_void_p(sp))
-        wl.compare_all(ctypes.c_void_p(sp))
-        for i, (W, q, s, qs, ss) in enumerate(wl.items):
-            host_q[i].copy_(q, non_blocking=True)
-            host_s[i].copy_(s, non_blocking=True)
-        host_r.copy_(wl.results, non_blocking=True)
+        for c, (i0, i1) in enumerate(chunks):
+            if done_k[c] is not None:
+                s_in.wait_event(done_k[c])
+            with torch.cuda.stream(s_in):
+                for i in range(i0, i1):
+                    wl.items[i][0].copy_(host_w[i], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+            s_k.wait_event(ev_in)
+            if done_out[c] is not None:
+                s_k.wait_event(done_out[c])
+            sk = ctypes.c_void_p(s_k.cuda_stream)
+            st = wl.L.mx_quantize_multi(ctypes.cast(qarrs[c], ctypes.c_void_p), i1 - i0, 1 | 4, sk)
+            if st:
+                raise RuntimeError(f"mx_quantize_multi failed: {st}")
+            st = wl.L.mx_grid_equal_multi(ctypes.cast(parrs[c], ctypes.c_void_p), 2 * (i1 - i0),
+                                          ctypes.c_void_p(wl.results[0, 2 * i0:].data_ptr()),
+                                          ctypes.c_void_p(wl.results[1, 2 * i0:].data_ptr()), sk)
+            if st:
+                raise RuntimeError(f"mx_grid_equal_multi failed: {st}")
+            done_k[c] = torch.cuda.Event()
+            done_k[c].record(s_k)
+            s_out.wait_event(done_k[c])
+            with torch.cuda.stream(s_out):
+                for i in range(i0, i1):
+                    host_q[i].copy_(wl.items[i][1], non_blocking=True)
+                    host_s[i].copy_(wl.items[i][2], non_blocking=True)
+                for row in range(2):
+                    host_r[row, 2 * i0:2 * i1].copy_(wl.results[row, 2 * i0:2 * i1], non_blocking=True)
+            done_out[c] = torch.cuda.Event()
+            done_out[c].record(s_out)
 
     one_step()
     torch.cuda.synchronize()
     steps = max(1, min(args.steps, 3))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(s_in)
     for _ in range(steps):
         one_step()
-    e1.record(stream)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     ok = int(host_r[0].sum()) == 0
     del host_w, host_q, host_s
     return {"value": round(wl.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 2), "steps": steps, "grid_equal": ok}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 2), "steps": steps, "grid_equal": ok,
+            "pipeline": f"{len(chunks)} chunks of <= {E2E_CHUNK} tensors on 3 streams (copy in, kernels, copy out)"}
 
 
 def aggregate_e2e(pg, local: dict, world: int, bytes_per_rank_step: int, device="cuda") -> dict:
@@ -491,6 +533,41 @@ def time_gpu(fn, reps, flush_buf, stream):
     return statistics.median(times)
 
 
+def device_status() -> dict:
+    """Reads and clears libmx's device status word after a timed region (synchronizes). A set bit
+    means some launch stopped early (an expired bounded wait, bad grouped offsets), so the time
+    beside it does not measure the whole computation: the line is then marked invalid."""
+    from mxfp8_block_scaled_07_b200 import mx
+
+    bits = mx.device_error()
+    return {"device_error": bits, "invalid": True} if bits else {"device_error": 0}
+
+
+def scaled_mm_fn(qa, sa, qb, sb):
+    """cuBLAS MXFP8 GEMM through torch `scaled_mm` (BlockWise1x32 scales in the SWIZZLE_32_4_4
+    layout) on this library's bytes and swizzled scales, BF16 out; None if torch lacks the path."""
+    import torch
+    import torch.nn.functional as F
+
+    try:
+        fa, fb = qa.view(torch.float8_e4m3fn), qb.view(torch.float8_e4m3fn).t()
+        ea, eb = sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu)
+        return lambda: F.scaled_mm(fa, fb, ea, F.ScalingType.BlockWise1x32, eb, F.ScalingType.BlockWise1x32,
+                                   swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                                   output_dtype=torch.bfloat16)
+    except (AttributeError, TypeError):
+        return None
+
+
+def cublas_line(fn, flops, reps, flush, stream) -> dict:
+    try:
+        fn()
+        ms = time_gpu(fn, reps, flush, stream)
+        return {"cublas_mxfp8_tflops": round(flops / (ms * 1e-3) / 1e12, 1), "cublas_ms": round(ms, 4)}
+    except (RuntimeError, TypeError, NotImplementedError) as e:
+        return {"cublas_mxfp8_tflops": None, "cublas_note": f"torch scaled_mm MXFP8 unavailable: {type(e).__name__}"}
+
+
 def guarded(fn):
     """A characterization line that fails reports its error in the JSON line instead of taking
     the headline measurement down with it."""
@@ -513,13 +590,21 @@ def run_secondary(device, peaks, reps=10):
            "fp8_peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
            "spec_fp8_tflops": 4500.0}
 
-    def add_gemm(name, flops, fn):
+    def add_gemm(name, flops, fn, lib_fn=None):
         for _ in range(2):
             fn()
+        mx.device_error()                     # clear before the timed launches
         ms = time_gpu(fn, reps, flush, stream)
         tf = flops / (ms * 1e-3) / 1e12
-        out["gemm"].append({"workload": name, "tflops": round(tf, 1), "ms": round(ms, 4),
-                            "frac_of_fp8_peak": round(tf / fp8_peak, 3), "frac_of_spec_4500": round(tf / 4500.0, 3)})
+        rec = {"workload": name, "tflops": round(tf, 1), "ms": round(ms, 4),
+               "frac_of_fp8_peak": round(tf / fp8_peak, 3), "frac_of_spec_4500": round(tf / 4500.0, 3)}
+        rec.update(device_status())
+        if lib_fn is not None:
+            lib = cublas_line(lib_fn, flops, reps, flush, stream)
+            rec.update(lib)
+            if lib.get("cublas_mxfp8_tflops"):
+                rec["mx_over_cublas"] = round(tf / lib["cublas_mxfp8_tflops"], 3)
+        out["gemm"].append(rec)
 
     def add_quant(name, x, row, col):
         bufs = mx.quantize(x, row, col, swizzle=True)
@@ -527,10 +612,13 @@ def run_secondary(device, peaks, reps=10):
         nbytes = M * K * 2 + (M * K + bufs[1].numel() if row else 0) + (M * K + bufs[3].numel() if col else 0)
         fn = lambda: mx.quantize(x, row, col, swizzle=True, out=bufs)
         fn()
+        mx.device_error()
         ms = time_gpu(fn, reps, flush, stream)
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out["quantize"].append({"workload": name, "gbs": round(gbs, 1), "ms": round(ms, 4),
-                                "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)})
+        rec = {"workload": name, "gbs": round(gbs, 1), "ms": round(ms, 4),
+               "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        rec.update(device_status())
+        out["quantize"].append(rec)
 
     # Dense forward linear (Table 5 micro-batch token counts) against gate_up.
     W = synth.sync_weight(0, 2, device=device)
@@ -541,7 +629,7 @@ def run_secondary(device, peaks, reps=10):
         qx, sx, _, _ = mx.quantize(X, True, False)
         C = torch.empty((M, W.shape[0]), dtype=torch.bfloat16, device=device)
         add_gemm(f"fwd {M}x24576x4096 bf16-out", 2.0 * M * W.shape[0] * W.shape[1],
-                 lambda: mx.gemm(qx, sx, qw, sw, out=C))
+                 lambda: mx.gemm(qx, sx, qw, sw, out=C), scaled_mm_fn(qx, sx, qw, sw))
         del X, qx, sx, C
     del W, qw, sw
     # Update micro-batch (12288 tokens): row + col quantization, fprop / dgrad / wgrad.
@@ -554,9 +642,12 @@ def run_secondary(device, peaks, reps=10):
     Y = torch.empty((T, O), dtype=torch.bfloat16, device=device)
     dX = torch.empty((T, H), dtype=torch.bfloat16, device=device)
     dW = torch.empty((O, H), dtype=torch.bfloat16, device=device)
-    add_gemm("update fprop 12288x12288x4096", 2.0 * T * O * H, lambda: mx.gemm(qx[0], qx[1], qwu[0], qwu[1], out=Y))
-    add_gemm("update dgrad 12288x4096x12288", 2.0 * T * H * O, lambda: mx.gemm(qd[0], qd[1], qwu[2], qwu[3], out=dX))
-    add_gemm("update wgrad 12288x4096x12288", 2.0 * O * H * T, lambda: mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW))
+    add_gemm("update fprop 12288x12288x4096", 2.0 * T * O * H, lambda: mx.gemm(qx[0], qx[1], qwu[0], qwu[1], out=Y),
+             scaled_mm_fn(qx[0], qx[1], qwu[0], qwu[1]))
+    add_gemm("update dgrad 12288x4096x12288", 2.0 * T * H * O, lambda: mx.gemm(qd[0], qd[1], qwu[2], qwu[3], out=dX),
+             scaled_mm_fn(qd[0], qd[1], qwu[2], qwu[3]))
+    add_gemm("update wgrad 12288x4096x12288", 2.0 * O * H * T, lambda: mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW),
+             scaled_mm_fn(qd[2], qd[3], qx[2], qx[3]))
     del X, Wu, dY, qx, qwu, qd, Y, dX, dW
     # MoE layer: grouped gate_up and down.
     counts, Xp, Hh, W1, W2 = synth.moe_inputs(device=device)
@@ -611,8 +702,10 @@ def run_secondary(device, peaks, reps=10):
     qbi, sbi, _, _ = mx.quantize(W1i, True, False)
     qbi = qbi.reshape(G, N2, K)
     hq = mx.grouped_gemm_swiglu_quant(qa, sa, qbi, sbi, offs, counts)
+    mx.device_error()
     fused_ms = time_gpu(lambda: mx.grouped_gemm_swiglu_quant(qa, sa, qbi, sbi, offs, counts, out=hq), reps, flush,
                         stream)
+    fused_status = device_status()
     qb, sb, _, _ = mx.quantize(W1.reshape(G * N2, K), True, False)
     qb = qb.reshape(G, N2, K)
     C = torch.empty((rows, N2), dtype=torch.bfloat16, device=device)
@@ -633,7 +726,7 @@ def run_secondary(device, peaks, reps=10):
         "fused_ms": round(fused_ms, 4), "fused_tflops": round(flops / (fused_ms * 1e-3) / 1e12, 1),
         "unfused_ms": round(unfused_ms, 4),
         "unfused": "mx_grouped_gemm (BF16 out) + torch SwiGLU + mx_quantize + mx_swizzle_scales",
-        "speedup": round(unfused_ms / fused_ms, 3)}
+        "speedup": round(unfused_ms / fused_ms, 3), **fused_status}
     del qa, sa_raw, sa, W1i, qbi, sbi, hq, qb, sb, C, hbuf, hs
     del Xp, Hh, W1, W2
     torch.cuda.synchronize()
@@ -660,8 +753,11 @@ def run_library_gemm_peak(device, reps=10):
     C = torch.empty((n, n), dtype=torch.bfloat16, device=device)
     flops = 2.0 * n * n * n
     out = {"shape": "8192x8192x8192 bf16-out"}
+    mx.gemm(qa, sa, qb, sb, out=C)
+    mx.device_error()
     ms = time_gpu(lambda: mx.gemm(qa, sa, qb, sb, out=C), reps, flush, stream)
     out["mx_gemm_tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    out.update(device_status())
     try:
         fa, fb = qa.view(torch.float8_e4m3fn), qb.view(torch.float8_e4m3fn).t()
         ea, eb = sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu)
@@ -679,16 +775,40 @@ def run_library_gemm_peak(device, reps=10):
 
 
 BREAKEVEN_TOKENS = (1312, 2592, 5216, 10304)   # 1.3k / 2.6k / 5.2k / 10.3k rounded to multiples of 32
+BREAKEVEN_PASSES = 3
 
 
-def run_breakeven(device, reps=20):
+def fit_line(xs, ys):
+    """Least-squares t = delta + c * x; returns (delta, c)."""
+    n = len(xs)
+    mx_, my = sum(xs) / n, sum(ys) / n
+    c = sum((x - mx_) * (y - my) for x, y in zip(xs, ys)) / sum((x - mx_) ** 2 for x in xs)
+    return my - c * mx_, c
+
+
+def breakeven_fit(points):
+    """The pages' stage cost model t = delta + c * tokens fitted per path over one sweep, and the
+    break-even tokens per micro-batch m* = (delta_mxfp8 - delta_bf16) / (c_bf16 - c_mxfp8)."""
+    xs = [p["tokens"] for p in points]
+    d_b, c_b = fit_line(xs, [p["bf16_ms"] for p in points])
+    d_m, c_m = fit_line(xs, [p["mxfp8_ms"] for p in points])
+    dd, dc = d_m - d_b, c_b - c_m
+    return {"bf16": {"delta_ms": round(d_b, 4), "c_us_per_token": round(c_b * 1e3, 5)},
+            "mxfp8": {"delta_ms": round(d_m, 4), "c_us_per_token": round(c_m * 1e3, 5)},
+            "delta_delta_ms": round(dd, 4), "delta_c_us_per_token": round(dc * 1e3, 5),
+            "m_star_tokens": (round(dd / dc, 1) if dc > 0 else None)}
+
+
+def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
     """Kernel-level fixed cost and per-token cost of one update micro-batch of a Qwen3-8B linear
     (W 12288 x 4096, the TP-2 gate_up shard): BF16 (cuBLAS fprop, dgrad, wgrad) against MXFP8
     (quantize X and dY row+col with the scale layout, then the three MXFP8 GEMMs), each micro-batch
-    one CUDA graph, L2 flushed before each replay. Fits t = delta + c * tokens per path (the pages'
-    stage cost model, Table 7) and reports the break-even tokens per micro-batch m* =
-    (delta_mxfp8 - delta_bf16) / (c_bf16 - c_mxfp8). The weight's own quantization happens once
-    per optimizer step, not per micro-batch, and is reported beside the fit."""
+    one CUDA graph, L2 flushed before each replay. The sweep over token counts is repeated `passes`
+    times, interleaved (every graph of a pass before the next pass), and the pages' stage cost
+    model t = delta + c * tokens (Table 7) is fitted per pass and path; m* = (delta_mxfp8 -
+    delta_bf16) / (c_bf16 - c_mxfp8) is reported per pass, with the fit of the per-point medians
+    and the spread. The weight's own quantization happens once per optimizer step, not per
+    micro-batch, and is reported beside the fit."""
     import torch
 
     from mxfp8_block_scaled_07_b200 import mx, synth
@@ -699,7 +819,8 @@ def run_breakeven(device, reps=20):
     W = synth.normal_bf16((O, H), std=0.02, seed=61, device=device)
     qw = mx.quantize(W, True, True)
     wq_ms = time_gpu(lambda: mx.quantize(W, True, True, out=qw), reps, flush, torch.cuda.current_stream())
-    rows = []
+    graphs = []               # (tokens, path, graph), buffers kept alive in `keep`
+    keep = []
     for T in BREAKEVEN_TOKENS:
         X = synth.normal_bf16((T, H), std=1.0, seed=62, device=device)
         dY = synth.normal_bf16((T, O), std=1e-3, seed=63, device=device)
@@ -708,20 +829,20 @@ def run_breakeven(device, reps=20):
         dW = torch.empty((O, H), dtype=torch.bfloat16, device=device)
         qx = mx.quantize(X, True, True)
         qd = mx.quantize(dY, True, True)
+        keep.append((X, dY, Y, dX, dW, qx, qd))
 
-        def bf16_step():
+        def bf16_step(X=X, dY=dY, Y=Y, dX=dX, dW=dW):
             torch.matmul(X, W.t(), out=Y)
             torch.matmul(dY, W, out=dX)
             torch.matmul(dY.t(), X, out=dW)
 
-        def mxfp8_step():
+        def mxfp8_step(X=X, dY=dY, Y=Y, dX=dX, dW=dW, qx=qx, qd=qd):
             mx.quantize(X, True, True, out=qx)
             mx.quantize(dY, True, True, out=qd)
             mx.gemm(qx[0], qx[1], qw[0], qw[1], out=Y)
             mx.gemm(qd[0], qd[1], qw[2], qw[3], out=dX)
             mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW)
 
-        times = {}
         for name, fn in (("bf16", bf16_step), ("mxfp8", mxfp8_step)):
             with torch.cuda.stream(stream):
                 fn()                                  # warm-up outside capture
@@ -729,33 +850,41 @@ def run_breakeven(device, reps=20):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
-            times[name] = time_gpu(g.replay, reps, flush, torch.cuda.current_stream())
-            del g
-        rows.append({"tokens": T, "bf16_ms": round(times["bf16"], 4), "mxfp8_ms": round(times["mxfp8"], 4)})
-        del X, dY, Y, dX, dW, qx, qd
+            graphs.append((T, name, g))
     torch.cuda.synchronize()
+    mx.device_error()
+    per_pass = []
+    for _ in range(passes):
+        t = {}
+        for T, name, g in graphs:
+            t[(T, name)] = time_gpu(g.replay, reps, flush, torch.cuda.current_stream())
+        per_pass.append([{"tokens": T, "bf16_ms": round(t[(T, "bf16")], 4), "mxfp8_ms": round(t[(T, "mxfp8")], 4)}
+                         for T in BREAKEVEN_TOKENS])
+    status = device_status()
+    del graphs, keep
+    torch.cuda.synchronize()
+    fits = [breakeven_fit(p) for p in per_pass]
+    med = [{"tokens": T,
+            "bf16_ms": round(statistics.median(p[i]["bf16_ms"] for p in per_pass), 4),
+            "mxfp8_ms": round(statistics.median(p[i]["mxfp8_ms"] for p in per_pass), 4)}
+           for i, T in enumerate(BREAKEVEN_TOKENS)]
+    out = {"linear": "W 12288x4096 (fprop, dgrad, wgrad per micro-batch)", "points": med, **breakeven_fit(med)}
+    ms_ = [f["m_star_tokens"] for f in fits if f["m_star_tokens"] is not None]
+    out["m_star_per_pass"] = [f["m_star_tokens"] for f in fits]
+    out["delta_delta_ms_per_pass"] = [f["delta_delta_ms"] for f in fits]
+    out["delta_c_us_per_token_per_pass"] = [f["delta_c_us_per_token"] for f in fits]
+    if ms_:
+        out["m_star_range"] = [min(ms_), max(ms_)]
+    out["weight_quantize_row_col_ms_per_step"] = round(wq_ms, 4)
+    out["timing"] = (f"one CUDA graph per micro-batch and path; {passes} interleaved passes, median of {reps} "
+                     "replays per point and pass, L2 flushed before each; points = per-point medians over passes")
+    out.update(status)
+    return out
 
-    def fit(ys):
-        xs = [r["tokens"] for r in rows]
-        n = len(xs)
-        mx_, my = sum(xs) / n, sum(ys) / n
-        c = sum((x - mx_) * (y - my) for x, y in zip(xs, ys)) / sum((x - mx_) ** 2 for x in xs)
-        return my - c * mx_, c
 
-    d_b, c_b = fit([r["bf16_ms"] for r in rows])
-    d_m, c_m = fit([r["mxfp8_ms"] for r in rows])
-    dd, dc = d_m - d_b, c_b - c_m
-    return {"linear": "W 12288x4096 (fprop, dgrad, wgrad per micro-batch)", "points": rows,
-            "bf16": {"delta_ms": round(d_b, 4), "c_us_per_token": round(c_b * 1e3, 5)},
-            "mxfp8": {"delta_ms": round(d_m, 4), "c_us_per_token": round(c_m * 1e3, 5)},
-            "delta_delta_ms": round(dd, 4), "delta_c_us_per_token": round(dc * 1e3, 5),
-            "m_star_tokens": (round(dd / dc, 1) if dc > 0 else None),
-            "weight_quantize_row_col_ms_per_step": round(wq_ms, 4),
-            "timing": "one CUDA graph per micro-batch and path, median of 20 replays, L2 flushed before each"}
-
-
-CASES = ("quant-gate-up", "quant-dy-rowcol", "gemm-fwd-10300", "gemm-update-fprop", "gemm-update-dgrad",
-         "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up")
+CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
+         "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up")
+SUBSET_LAYERS = 2      # quant-sync-subset: the first 2 layers' 8 weights (0.39 G elements, ~1.2 GB on the device)
 
 
 def run_case(name: str, reps: int):
@@ -769,6 +898,17 @@ def run_case(name: str, reps: int):
     dev = torch.device("cuda", 0)
     if name == "quant-gate-up":
         x = synth.sync_weight(0, 2, device=dev)
+        bufs = mx.quantize(x, True, False)
+        fn = lambda: mx.quantize(x, True, False, out=bufs)
+    elif name == "quant-sync-subset":
+        # The headline launch (mx_quantize_multi ROWWISE|SWIZZLE) over a subset of the 144 weights,
+        # for DRAM-traffic captures: per-element traffic scales to the full launch.
+        xs = [synth.sync_weight(layer, idx, device=dev) for layer in range(SUBSET_LAYERS) for idx in range(4)]
+        outs = mx.quantize_multi(xs, True, False, True)
+        fn = lambda: mx.quantize_multi(xs, True, False, True, outs=outs)
+        print(json.dumps({"case": name, "tensors": len(xs), "elements": int(sum(x.numel() for x in xs))}))
+    elif name == "quant-fwd-1300":
+        x = synth.fwd_activations(1300, device=dev)
         bufs = mx.quantize(x, True, False)
         fn = lambda: mx.quantize(x, True, False, out=bufs)
     elif name == "quant-dy-rowcol":
@@ -878,6 +1018,7 @@ def main():
         time.sleep(0.25)
     if pg is not None:
         pg.barrier()
+    headline_err = sum_over_ranks(pg, mx.device_error())     # any rank's status bits mark the run
     ms_local = t0.elapsed_time(t1) / args.steps
     quant_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
     cmp_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
@@ -905,6 +1046,10 @@ def main():
     cpu = None
     if not args.no_e2e:                  # every rank: the whole job's end-to-end step
         e2e = aggregate_e2e(pg, run_e2e(wl, args, device), world, wl.step_bytes)
+        e2e_err = mx.device_error()
+        if e2e_err:
+            e2e["device_error"] = e2e_err
+            e2e["invalid"] = True
     del wl
     torch.cuda.empty_cache()
     # Kernel characterization lines (one GPU's kernels) only in single-GPU runs: the other ranks
@@ -937,6 +1082,7 @@ def main():
             "gpu_launches": args.steps * SyncWorkload.LAUNCHES_PER_STEP,
             "clocks": clocks.summary(),
             "grid_equal_mismatches": mismatches,
+            "device_error": headline_err,
             "secondary": secondary,
         }
         print(json.dumps(line), flush=True)

@@ -74,7 +74,7 @@ int64_t mx_swizzled_scale_bytes(int64_t rows, int64_t kblocks);
  *   MX_COLWISE: q_col[K, M] = the rowwise quantization of x^T (blocks of 32 along M, stored
  *               K-major for the transposed GEMM operands of dgrad / wgrad) and s_col: raw
  *               [K, M/32] or swizzled (mx_swizzled_scale_bytes(K, M/32) bytes).
- * Requirements: K % 32 == 0; M % 32 == 0 if MX_COLWISE; ld_x >= K and ld_x % 8 == 0; at least
+ * Requirements: K % 32 == 0; M % 32 == 0 if MX_COLWISE; M, K < 2^31; ld_x >= K and ld_x % 8 == 0; at least
  * one of MX_ROWWISE / MX_COLWISE; the pointers of each requested direction non-NULL (others are
  * ignored); all pointers 16-byte aligned. M == 0 or K == 0 is a no-op.
  * Result is bit-exact to the rule in the header comment.
@@ -198,8 +198,8 @@ mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz,
  * s = 1; a block holding NaN or Inf takes s = NaN and codes sign|0x7F.
  *   x: BF16 [M, K] (device), row stride ld_x elements; q: [M, K] E4M3 codes (device, packed);
  *   scales: fp32 [ceil(M/128), ceil(K/128)] row-major (device).
- * Requirements: K % 32 == 0, ld_x >= K, ld_x % 8 == 0, x and q 16-byte aligned, scales 4-byte
- * aligned. M == 0 or K == 0 is a no-op (pointers may then be NULL).
+ * Requirements: K % 32 == 0, M, K < 2^31 (else MX_ERR_SHAPE), ld_x >= K, ld_x % 8 == 0, x and q
+ * 16-byte aligned, scales 4-byte aligned. M == 0 or K == 0 is a no-op (pointers may then be NULL).
  * Errors: MX_ERR_ARG, MX_ERR_SHAPE, MX_ERR_ALIGN as stated; MX_ERR_CUDA on a failed launch.
  */
 mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x, int pow2_scales, uint8_t* q,
@@ -212,6 +212,14 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
  * fp32 summation order only. Other values select 0.
  */
 void mx_set_gemm_variant(int variant);
+
+/*
+ * Selects the quantizer kernel behind later mx_quantize / mx_quantize_multi calls (process-wide):
+ * 0 (default) stages each 128 x 128 BF16 tile in shared memory with TMA loads running a few tiles
+ * ahead of the compute; 1 loads tiles into registers with a one-tile prefetch. Both produce the
+ * same bytes. Other values select 0.
+ */
+void mx_set_quantize_variant(int variant);
 
 /*
  * Byte comparison (abstract and Table 11: the synchronized sampler weights, scales and kernel
@@ -252,7 +260,9 @@ mx_status mx_device_error(uint32_t* bits);
 
 /*
  * Deadline of every bounded wait inside libmx kernels, in nanoseconds (default 2e9 = 2 s); 0
- * restores the default. Affects launches made after the call.
+ * restores the default. Affects launches made after the call. After a wait expires, a kernel still
+ * waits for its own copies and MMAs in flight before it exits; those drain waits take at least 1 s
+ * whatever this deadline is.
  */
 void mx_set_wait_timeout_ns(uint64_t ns);
 

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmx.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("libmx.cu",)]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quantize.cuh", "swizzle.cuh", "grid_equal.cuh", "gemm.cuh", "blockwise.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quantize.cuh", "quantize_tma.cuh", "swizzle.cuh", "grid_equal.cuh", "gemm.cuh", "blockwise.cuh")] + [
     os.path.join(ROOT, "include", "mx.h")
 ]
 

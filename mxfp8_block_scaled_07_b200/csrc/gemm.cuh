@@ -643,6 +643,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    uint32_t* issued_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc + 8);   // this CTA's operand fills
     int32_t* off = reinterpret_cast<int32_t*>(smem + L::kGroups);
     int32_t* pm128 = off + (kMaxGroups + 1);
     int32_t* pm256 = pm128 + (kMaxGroups + 1);
@@ -715,15 +716,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
         }
-        if (!ok && leader) {
-            // Wait for the copies still in flight (both CTAs' loads count on the leader's barriers).
-            int s = stage;
-            uint32_t p = phase;
-            for (int i = 0; i < min(issued, S); ++i) {
-                if (--s < 0) { s = S - 1; p ^= 1u; }
-                mbar_wait_drain(&full[s], p, a.timeout_ns);
-            }
-        }
+        if (lane == 0) *issued_slot = static_cast<uint32_t>(issued);   // read by the leader's drain
     } else if (warp == 1) {
         if (leader) {
             // ---------------- MMA issuer (leader CTA, for both) ----------------
@@ -794,8 +787,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     // Neither CTA leaves (or frees TMEM) while the pair still has MMAs, copies or signals in flight.
+    // Past the first cluster barrier no role of either CTA issues anything. Both CTAs' operand
+    // copies complete on the leader's `full` barriers; after an expired wait the two producers may
+    // have stopped at different fills, so the leader drains the last S fills either CTA issued:
+    // for a fill only one CTA issued it supplies the missing half of the stage's transaction count
+    // (the bytes that were never requested, or its own arrival for the peer's bytes) and waits for
+    // the copies that were. On the normal path every phase has completed and these waits return
+    // at once.
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
+    if (leader && warp == 0 && lane == 0) {
+        const uint32_t mine = *issued_slot;
+        const uint32_t peer = ld_shared_cluster_u32(mapa_shared(smem_u32(issued_slot), 1));
+        const uint32_t hi = max(mine, peer);
+        for (uint32_t i = hi > static_cast<uint32_t>(S) ? hi - S : 0u; i < hi; ++i) {
+            uint64_t* bar = &full[i % S];
+            if (i >= mine)
+                mbar_arrive_expect_tx(bar, kPairStageBytes);    // the peer's copies only
+            else if (i >= peer)
+                mbar_complete_tx(bar, kPairStageBytes);         // the peer never requested its half
+            mbar_wait_drain(bar, (i / S) & 1u, a.timeout_ns);
+        }
+    }
     cluster_sync();
     if (warp == 1) {
         tc_fence_after();

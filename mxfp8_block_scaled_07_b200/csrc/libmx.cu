@@ -16,6 +16,7 @@
 #include "grid_equal.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
+#include "quantize_tma.cuh"
 #include "swizzle.cuh"
 
 namespace mx {
@@ -47,6 +48,7 @@ struct DeviceInfo {
     int cc_major = 0;
     uint32_t* status = nullptr;
     int quant_blocks_per_sm[4] = {0, 0, 0, 0};
+    int qt_blocks_per_sm[4] = {0, 0, 0, 0};   // TMA-staged quantizer, by direction bits
     int ge_blocks_per_sm = 1;
     int pair_clusters[2] = {0, 0};    // co-resident 2-CTA clusters of the pair GEMM (dense, grouped)
     bool ok = false;
@@ -76,6 +78,8 @@ int max_pair_clusters(K kernel, int smem, int sms) {
 
 // GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
 std::atomic<int> g_gemm_variant{0};
+// Quantizer selection: 0 = TMA-staged tiles (default), 1 = register-staged tiles.
+std::atomic<int> g_quant_variant{0};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -90,6 +94,22 @@ int quant_occupancy() {
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_rowcol_kernel<ROW, kQMaxTensors>, kQThreads, 0);
     return n > 0 ? n : 1;
+}
+
+// Opts the TMA-staged quantizer (both tensor-count instantiations) into its dynamic shared memory
+// and returns its resident CTAs per SM.
+template <bool ROW, bool COL>
+bool qt_setup(int* blocks) {
+    if (cudaFuncSetAttribute(quantize_tma_kernel<ROW, COL, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kQtSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(quantize_tma_kernel<ROW, COL, kQtMaxTensors>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kQtSmemBytes) != cudaSuccess)
+        return false;
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_tma_kernel<ROW, COL, kQtMaxTensors>, kQThreads,
+                                                  kQtSmemBytes);
+    *blocks = n > 0 ? n : 1;
+    return true;
 }
 
 // Per-device facts, queried once with that device current.
@@ -114,6 +134,9 @@ const DeviceInfo* device_info() {
         if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
         d.quant_blocks_per_sm[2] = quant_occupancy<false>();
         d.quant_blocks_per_sm[3] = quant_occupancy<true>();
+        if (!qt_setup<true, false>(&d.qt_blocks_per_sm[1]) || !qt_setup<false, true>(&d.qt_blocks_per_sm[2]) ||
+            !qt_setup<true, true>(&d.qt_blocks_per_sm[3]))
+            return nullptr;
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.ge_blocks_per_sm, grid_equal_kernel<kGeMaxPairs>,
                                                       kGeThreads, 0);
         if (d.ge_blocks_per_sm < 1) d.ge_blocks_per_sm = 1;
@@ -291,6 +314,7 @@ namespace {
 mx_status check_quant_tensor(const mx_quant_tensor& t, bool row, bool col, bool* empty) {
     if (t.M < 0 || t.K < 0) return MX_ERR_ARG;
     if (t.K % 32 != 0 || (col && t.M % 32 != 0)) return MX_ERR_SHAPE;
+    if (t.M >= (int64_t(1) << 31) || t.K >= (int64_t(1) << 31)) return MX_ERR_SHAPE;
     *empty = (t.M == 0 || t.K == 0);
     if (*empty) return MX_OK;   // empty tensors may carry null pointers
     if (!t.x || (row && (!t.q_row || !t.s_row)) || (col && (!t.q_col || !t.s_col))) return MX_ERR_ARG;
@@ -335,6 +359,54 @@ mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceI
     return launched();
 }
 
+// Tensor map of a BF16 input [M, K] (row stride ld_x elements) in 64-column x 128-row boxes with the
+// 128-byte swizzle the TMA-staged quantizer reads; out-of-range elements arrive as zeros.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t M, int64_t K, int64_t ld_x) {
+    if (!encode_fn()) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NT>
+bool add_qt_tensor(QuantTmaArgs<NT>& a, const mx_quant_tensor& t) {
+    const int i = a.n;
+    if (!make_tmap_bf16(&a.map[i], t.x, t.M, t.K, t.ld_x)) return false;
+    QtTensor& q = a.t[i];
+    q.q_row = t.q_row;
+    q.s_row = t.s_row;
+    q.q_col = t.q_col;
+    q.s_col = t.s_col;
+    q.M = static_cast<int32_t>(t.M);
+    q.K = static_cast<int32_t>(t.K);
+    q.tiles_m = static_cast<int32_t>(ceil_div(t.M, kQTile));
+    q.tiles_k = static_cast<int32_t>(ceil_div(t.K, kQTile));
+    q.vec32 = reinterpret_cast<uintptr_t>(t.q_row) % 32 == 0;
+    q.col_vec32 = reinterpret_cast<uintptr_t>(t.q_col) % 32 == 0;
+    q.tile_start = a.total_tiles;
+    a.total_tiles += int64_t(q.tiles_m) * q.tiles_k;
+    ++a.n;
+    return true;
+}
+
+template <int NT>
+mx_status launch_qt(const QuantTmaArgs<NT>& a, bool row, bool col, const DeviceInfo* d, mx_stream stream) {
+    if (a.total_tiles == 0) return MX_OK;
+    const int which = (row ? 1 : 0) | (col ? 2 : 0);
+    const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->qt_blocks_per_sm[which]);
+    if (row && col)
+        quantize_tma_kernel<true, true, NT><<<grid, kQThreads, kQtSmemBytes, stream>>>(a);
+    else if (row)
+        quantize_tma_kernel<true, false, NT><<<grid, kQThreads, kQtSmemBytes, stream>>>(a);
+    else
+        quantize_tma_kernel<false, true, NT><<<grid, kQThreads, kQtSmemBytes, stream>>>(a);
+    return launched();
+}
+
 template <int NP>
 void add_pair(CmpArgs<NP>& g, const uint8_t* a, const uint8_t* b, int64_t nbytes) {
     CmpPair& p = g.p[g.n++];
@@ -372,6 +444,16 @@ mx_status mx_quantize(const void* x, int64_t M, int64_t K, int64_t ld_x, int fla
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
+    if (g_quant_variant.load() == 0) {
+        QuantTmaArgs<1> a;
+        a.n = 0;
+        a.swz = swz;
+        a.total_tiles = 0;
+        a.err = d->status;
+        a.timeout_ns = g_timeout_ns.load();
+        if (!add_qt_tensor(a, t)) return MX_ERR_CUDA;
+        return launch_qt(a, row, col, d, stream);
+    }
     QuantArgs<1> a;
     a.n = 0;
     a.swz = swz;
@@ -392,6 +474,23 @@ mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags
     if (n == 0) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
+    if (g_quant_variant.load() == 0) {
+        static thread_local QuantTmaArgs<kQtMaxTensors> a;   // ~30 KB: kept off the stack
+        for (int64_t i0 = 0; i0 < n; i0 += kQtMaxTensors) {
+            a.n = 0;
+            a.swz = swz;
+            a.total_tiles = 0;
+            a.err = d->status;
+            a.timeout_ns = g_timeout_ns.load();
+            for (int64_t i = i0; i < std::min<int64_t>(n, i0 + kQtMaxTensors); ++i) {
+                const mx_quant_tensor& t = tensors[i];
+                if (t.M > 0 && t.K > 0 && !add_qt_tensor(a, t)) return MX_ERR_CUDA;
+            }
+            if (a.n == 0) continue;
+            if (mx_status st = launch_qt(a, row, col, d, stream)) return st;
+        }
+        return MX_OK;
+    }
     static thread_local QuantArgs<kQMaxTensors> a;   // ~14 KB: kept off the stack
     for (int64_t i0 = 0; i0 < n; i0 += kQMaxTensors) {
         a.n = 0;
@@ -640,7 +739,7 @@ mx_status mx_grouped_gemm_swiglu_quant(const uint8_t* qa, const uint8_t* sa_swz,
 mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x, int pow2_scales, uint8_t* q,
                                float* scales, mx_stream stream) {
     if (M < 0 || K < 0) return MX_ERR_ARG;
-    if (K % 32 != 0) return MX_ERR_SHAPE;
+    if (K % 32 != 0 || M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return MX_ERR_SHAPE;
     if (M == 0 || K == 0) return MX_OK;                // empty: pointers may be NULL
     if (!x || !q || !scales) return MX_ERR_ARG;
     if (ld_x < K) return MX_ERR_SHAPE;
@@ -667,5 +766,7 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
 }
 
 void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
+
+void mx_set_quantize_variant(int variant) { g_quant_variant.store(variant == 1 ? 1 : 0); }
 
 }  // extern "C"

@@ -63,14 +63,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Same, but ignores `abort` (used while draining in-flight copies before exit).
+// Lower bound of the deadline of a drain wait, independent of the (possibly very short) deadline of
+// the ordinary waits: copies and MMAs in flight complete in microseconds, and a CTA must not exit
+// (or free TMEM) before they have.
+constexpr uint64_t kDrainFloorNs = 1000000000ull;
+
+// Same, but ignores `abort` (used while draining in-flight copies and MMAs before exit). Waits at
+// least kDrainFloorNs.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
     const uint32_t a = smem_u32(bar);
+    const uint64_t limit = timeout_ns > kDrainFloorNs ? timeout_ns : kDrainFloorNs;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > timeout_ns) return false;
+        if (globaltimer_ns() - t0 > limit) return false;
     }
     return true;
+}
+
+// Single-thread forms used on the drain path: one arrival that expects `bytes` more, and a
+// completion of `bytes` without data (for copies that were never issued).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
 // ---- shared / global vector access, tensor-map prefetch ---------------------------------------
@@ -174,6 +190,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit load from a shared::cluster address (possibly in the peer CTA).
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
 }
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {

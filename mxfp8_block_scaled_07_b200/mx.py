@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.mx_set_wait_timeout_ns.restype = None
     L.mx_set_gemm_variant.argtypes = [I32]
     L.mx_set_gemm_variant.restype = None
+    L.mx_set_quantize_variant.argtypes = [I32]
+    L.mx_set_quantize_variant.restype = None
     L.mx_diag_expired_wait.argtypes = [P]
     L.mx_diag_expired_wait.restype = I32
     _lib = L
@@ -299,3 +301,11 @@ GEMM_PAIR, GEMM_SINGLE = 0, 1
 def set_gemm_variant(variant: int):
     """0: CTA-pair GEMM kernel (default); 1: single-CTA kernel."""
     lib().mx_set_gemm_variant(int(variant))
+
+
+QUANT_TMA, QUANT_REGISTERS = 0, 1
+
+
+def set_quantize_variant(variant: int):
+    """0: TMA-staged quantizer (default); 1: register-staged quantizer. Same bytes either way."""
+    lib().mx_set_quantize_variant(int(variant))

@@ -37,3 +37,14 @@ def gemm_variant(request):
     mx.set_gemm_variant(request.param)
     yield request.param
     mx.set_gemm_variant(0)
+
+
+@pytest.fixture(params=[0, 1], ids=["tma", "regs"])
+def quant_variant(request):
+    """Runs a quantizer test with the TMA-staged kernel (0, the default) and the register-staged
+    kernel (1)."""
+    from mxfp8_block_scaled_07_b200 import mx
+
+    mx.set_quantize_variant(request.param)
+    yield request.param
+    mx.set_quantize_variant(0)

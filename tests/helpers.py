@@ -36,3 +36,27 @@ def assert_gemm_close(c_gpu, ref, abs_sum, bf16: bool, what=""):
             f"ref {ref[tuple(i)]!r} bound {bound[tuple(i)] if np.ndim(bound) else bound!r}")
     ratio = np.where(abs_sum > 0, err / np.maximum(abs_sum, 1e-300), 0.0)
     return float(ratio.max()) if ratio.size else 0.0
+
+
+def check_sampled_rows(x_dev: torch.Tensor, q_dev: torch.Tensor, s_dev: torch.Tensor, rows, group_rows=None,
+                       swizzled: bool = True, what: str = ""):
+    """Rowwise quantization of the CUDA tensor x_dev, checked against the oracle on the sampled
+    rows: E4M3 codes, and the scale bytes either raw ([rows, K/32]) or at their positions in the
+    (grouped) tensor-core layout, whose pad bytes must all be 0. The oracle quantizes the BF16 rows
+    itself; nothing of the GPU result reaches it."""
+    rows = np.unique(np.asarray(rows, np.int64))
+    M, K = x_dev.shape
+    r_dev = torch.from_numpy(rows).to(x_dev.device)
+    qo, so = oracle.quantize_rowwise(x_dev[r_dev].cpu())
+    q = to_np(q_dev[r_dev])
+    bad = np.argwhere(q != qo)
+    assert bad.size == 0, f"{what}: {len(bad)} code bytes differ; first at row {rows[bad[0][0]]} col {bad[0][1]}"
+    s_np = to_np(s_dev)
+    if not swizzled:
+        assert np.array_equal(s_np[rows], so), f"{what}: raw scales"
+        return
+    pos = scale_positions(M, K // 32, group_rows)
+    assert np.array_equal(s_np.reshape(-1)[pos[rows]], so), f"{what}: scale bytes in the layout"
+    pad = np.ones(s_np.size, bool)
+    pad[pos.reshape(-1)] = False
+    assert not s_np.reshape(-1)[pad].any(), f"{what}: nonzero pad bytes in the scale layout"

@@ -30,3 +30,21 @@ def test_warmup_below_three_is_rejected():
     out = subprocess.run([sys.executable, "bench.py", "--steps", "1", "--warmup", "2"], cwd=ROOT,
                          capture_output=True, text=True, timeout=120)
     assert out.returncode != 0 and "--warmup" in out.stderr
+
+
+def test_breakeven_fit_recovers_the_stage_cost_model():
+    """t = delta + c * tokens per path (Table 7's stage cost model), m* = d_delta / d_c."""
+    import pytest
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    pts = [{"tokens": T, "bf16_ms": 0.020 + 2.0e-4 * T, "mxfp8_ms": 0.030 + 1.3e-4 * T}
+           for T in bench.BREAKEVEN_TOKENS]
+    f = bench.breakeven_fit(pts)
+    assert f["bf16"]["delta_ms"] == pytest.approx(0.020, abs=1e-4)
+    assert f["mxfp8"]["c_us_per_token"] == pytest.approx(0.13, rel=1e-3)
+    assert f["m_star_tokens"] == pytest.approx(0.010 / 7.0e-5, rel=1e-3)
+    # No saving per token: no break-even.
+    flat = [{"tokens": T, "bf16_ms": 1.0, "mxfp8_ms": 2.0} for T in bench.BREAKEVEN_TOKENS]
+    assert bench.breakeven_fit(flat)["m_star_tokens"] is None

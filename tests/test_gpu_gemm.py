@@ -135,7 +135,7 @@ def cols_of(t_dev):
     return lambda idx: t_dev[:, torch.from_numpy(np.asarray(idx)).to(t_dev.device)].t().contiguous().cpu()
 
 
-@pytest.mark.parametrize("M", [1300, 10300])
+@pytest.mark.parametrize("M", synth.FWD_TOKENS)
 def test_fwd_linear_full_size_sampled(M):
     # Qwen3-8B forward linear: X[M, 4096] (lognormal channels) . W_gate_up[24576, 4096]^T, BF16 out.
     X = synth.fwd_activations(M, device="cuda")
@@ -161,3 +161,53 @@ def test_update_step_full_size_sampled():
     sampled_check(rows_of(X), rows_of(W), Y, np.array([5, 12287]), np.array([0, 12287]), 48, True, "fprop")
     sampled_check(rows_of(dY), cols_of(W), dX, np.array([0, 9000]), np.array([17, 4095]), 48, True, "dgrad")
     sampled_check(cols_of(dY), cols_of(X), dW, np.array([1, 12287]), np.array([0, 4095]), 48, True, "wgrad")
+
+
+def test_update_step_fp32_out_long_k():
+    """The update step's K = 12 288 contractions (dgrad over the output features, wgrad over the
+    tokens) with fp32 output, where the 2^-8 term of the BF16 bound cannot hide the accumulator:
+    every sampled element within 1e-5 * sum_k |a_k b_k| of the fp64 oracle. Also the forward
+    K = 4096 product in fp32. Prints the worst err / sum|ab| seen."""
+    X, W, dY = synth.update_inputs(device="cuda")
+    _, _, qx_c, sx_c = mx.quantize(X, False, True)
+    qw_r, sw_r, qw_c, sw_c = mx.quantize(W, True, True)
+    qd_r, sd_r, qd_c, sd_c = mx.quantize(dY, True, True)
+    qx_r, sx_r, _, _ = mx.quantize(X, True, False)
+    dX = mx.gemm(qd_r, sd_r, qw_c, sw_c, out_dtype=torch.float32)      # K = 12288
+    dW = mx.gemm(qd_c, sd_c, qx_c, sx_c, out_dtype=torch.float32)      # K = 12288
+    Y = mx.gemm(qx_r, sx_r, qw_r, sw_r, out_dtype=torch.float32)       # K = 4096
+    torch.cuda.synchronize()
+    worst = {
+        "dgrad": sampled_check(rows_of(dY), cols_of(W), dX, np.array([3, 12287]), np.array([0, 4095]), 48, False,
+                               "dgrad fp32", seed=1),
+        "wgrad": sampled_check(cols_of(dY), cols_of(X), dW, np.array([0, 12287]), np.array([1, 4095]), 48, False,
+                               "wgrad fp32", seed=2),
+        "fprop": sampled_check(rows_of(X), rows_of(W), Y, np.array([0, 12287]), np.array([7, 12287]), 48, False,
+                               "fprop fp32", seed=3),
+    }
+    print("worst |c - ref| / sum|ab| (bound 1e-5):", {k: f"{v:.3e}" for k, v in worst.items()})
+    assert max(worst.values()) <= 1e-5
+
+
+def test_expired_waits_end_the_gemm_cleanly(gemm_variant):
+    """With a 1 ns deadline every wait that does not succeed at once expires: the kernel records
+    error bit 1, every role stops, in-flight copies and MMAs are drained (those drain waits keep a
+    floor of 1 s), TMEM is freed and the launch returns. The context stays usable: the next GEMM
+    under the default deadline is exact."""
+    M, N, K = 1024, 1024, 16384
+    A = synth.normal_bf16((M, K), seed=91)
+    B = synth.normal_bf16((N, K), seed=92)
+    qa, sa = gpu_operand(A.cuda())
+    qb, sb = gpu_operand(B.cuda())
+    torch.cuda.synchronize()
+    assert mx.device_error() == 0
+    mx.set_wait_timeout_ns(1)
+    try:
+        mx.gemm(qa, sa, qb, sb, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        bits = mx.device_error()
+    finally:
+        mx.set_wait_timeout_ns(0)
+    assert bits == 1
+    check_case(A[:256, :1024].contiguous(), B[:384, :1024].contiguous(), torch.float32, "after expired waits")
+    assert mx.device_error() == 0

@@ -37,26 +37,26 @@ def run_both(x_cpu: torch.Tensor, rowwise=True, colwise=False, ld_pad=0):
         assert np.array_equal(to_np(swz[3]), oracle.swizzle(sT)), "colwise swizzled scales"
 
 
-def test_pr1_operands_row_and_col():
+def test_pr1_operands_row_and_col(quant_variant):
     A, B = synth.pr1_inputs()
     run_both(A, True, True)
     run_both(B, True, True)
 
 
 @pytest.mark.parametrize("shape", [(1, 32), (33, 96), (130, 160), (256, 512), (300, 1056), (7, 4096), (129, 4128)])
-def test_rowwise_ragged_shapes(shape):
+def test_rowwise_ragged_shapes(shape, quant_variant):
     x = synth.normal_bf16(shape, std=0.5, seed=shape[0] * 7 + shape[1], outlier_frac=0.01, outlier_scale=100.0)
     run_both(x, True, False)
 
 
 @pytest.mark.parametrize("shape", [(32, 32), (64, 96), (160, 288), (384, 544), (96, 4096), (4096, 160)])
-def test_row_and_col_ragged_shapes(shape):
+def test_row_and_col_ragged_shapes(shape, quant_variant):
     x = synth.normal_bf16(shape, std=3.0, seed=shape[0] + shape[1], outlier_frac=0.01, outlier_scale=50.0)
     run_both(x, True, True)
     run_both(x, False, True)
 
 
-def test_strided_input():
+def test_strided_input(quant_variant):
     x = synth.normal_bf16((200, 320), seed=4)
     run_both(x, True, False, ld_pad=24)
     x = synth.normal_bf16((192, 320), seed=5)
@@ -64,12 +64,12 @@ def test_strided_input():
 
 
 @pytest.mark.parametrize("seed", [0, 1])
-def test_special_values_nan_inf_zero_subnormal(seed):
+def test_special_values_nan_inf_zero_subnormal(seed, quant_variant):
     x = synth.special_bf16((256, 1024), seed=seed)
     run_both(x, True, True)
 
 
-def test_every_bf16_pattern_in_blocks():
+def test_every_bf16_pattern_in_blocks(quant_variant):
     # All 65536 BF16 bit patterns, 32 to a block, in two arrangements (sorted: blocks of nearby
     # magnitude; shuffled: mixed magnitudes, so most elements sit far below their block's amax).
     bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
@@ -121,7 +121,7 @@ def test_update_step_columnwise_full_size_sampled():
 
 @pytest.mark.parametrize("rowwise,colwise", [(True, False), (True, True), (False, True)])
 @pytest.mark.parametrize("swizzle", [True, False])
-def test_quantize_multi_matches_oracle(rowwise, colwise, swizzle):
+def test_quantize_multi_matches_oracle(rowwise, colwise, swizzle, quant_variant):
     # Several tensors of mixed shapes (ragged, tiny, empty, strided) in one launch.
     shapes = [(256, 512), (32, 96), (160, 288), (0, 64), (384, 1056), (96, 32), (1024, 128)]
     xs = []
@@ -148,7 +148,7 @@ def test_quantize_multi_matches_oracle(rowwise, colwise, swizzle):
             assert np.array_equal(to_np(s_col), oracle.swizzle(sT) if swizzle else sT)
 
 
-def test_quantize_multi_more_tensors_than_one_launch_holds():
+def test_quantize_multi_more_tensors_than_one_launch_holds(quant_variant):
     # 400 small tensors: split over several launches inside one call.
     xs = [synth.normal_bf16((32 * (1 + i % 5), 64 * (1 + i % 3)), seed=100 + i) for i in range(400)]
     outs = mx.quantize_multi([x.cuda() for x in xs], True, False, True)

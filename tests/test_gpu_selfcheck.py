@@ -3,12 +3,23 @@
 Faults follow "End-to-End MXFP8 Reinforcement Learning on Blackwell", Table 10: F3 (the sampler's
 swizzled scale copy is left from the previous weights while its elements are fresh) and F4 (an
 in-place repack of the experts that keeps shape and dtype). A healthy sampler gives exactly 0
-mismatching output bytes; both faults give many. The relative error against a BF16 product of the
-synchronized weights is reported beside it (the pages' MoE probe: 0.05 healthy, 1.74 with F4).
+mismatching output bytes; both faults give many.
+
+Beside the byte comparison, the probe's relative error ||y - ref|| / ||ref|| is measured against two
+references computed by the CPU oracle from the same synchronized weights (the pages' MoE probe:
+0.05 healthy, 1.74 with F4):
+  - the oracle's MXFP8 GEMM of the learner's grid (fp64 over the oracle's own quantization of the
+    BF16 activations and weights): a healthy sampler differs from it only by the BF16 rounding of
+    the output and the GEMM tolerance, so <= 2^-8; a stale sampler by far more;
+  - the exact fp64 product of the BF16 activations and weights (a numpy matmul): a healthy sampler
+    is off by the MXFP8 quantization error (about 0.05, the pages' healthy figure).
 """
+import numpy as np
 import pytest
 import torch
 
+import oracle
+from helpers import to_np
 from mxfp8_block_scaled_07_b200 import mx, selfcheck, synth
 
 pytestmark = pytest.mark.gpu
@@ -25,6 +36,15 @@ def sampler_copy(w):
 
 def rel_err(y, ref):
     return float(((y.float() - ref).norm() / ref.norm()).item())
+
+
+def rel_err_np(y, ref):
+    y = np.asarray(y, np.float64)
+    return float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+
+
+def bf16_f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
 
 
 def test_dense_probe_healthy_and_stale_scales():
@@ -48,9 +68,27 @@ def test_dense_probe_healthy_and_stale_scales():
     cnt, first = selfcheck.probe_dense(x, w, q, s_old)
     torch.cuda.synchronize()
     assert int(cnt.item()) > 0 and int(first.item()) >= 0
-    stale = rel_err(mx.gemm(qx, sx, q, s_old), ref)
+    y_stale = mx.gemm(qx, sx, q, s_old)
+    stale = rel_err(y_stale, ref)
     assert stale > 2 * healthy
-    print(f"dense probe: relative error healthy {healthy:.4f}, stale scales {stale:.4f}")
+
+    # Against the oracle on sampled output rows: its MXFP8 GEMM of the learner's grid, and the
+    # exact product of the BF16 values.
+    rows = np.unique(np.concatenate([[0, T - 1], np.random.default_rng(5).integers(0, T, 22)]))
+    r_dev = torch.from_numpy(rows).cuda()
+    qx_o, sx_o = oracle.quantize_rowwise(x[r_dev].cpu())
+    qw_o, sw_o = oracle.quantize_rowwise(w.cpu())
+    ref_mx, _ = oracle.gemm(qx_o, sx_o, qw_o, sw_o)
+    exact = bf16_f64(x[r_dev]) @ bf16_f64(w).T
+    y_ok = to_np(mx.gemm(qx, sx, q, s)[r_dev].float())
+    y_bad = to_np(y_stale[r_dev].float())
+    e_ok, e_bad = rel_err_np(y_ok, ref_mx), rel_err_np(y_bad, ref_mx)
+    x_ok, x_bad = rel_err_np(y_ok, exact), rel_err_np(y_bad, exact)
+    assert e_ok <= 2.0 ** -8 and e_bad > 0.1
+    assert x_ok < 0.1 and x_bad > 2 * x_ok
+    print(f"dense probe: relative error healthy {healthy:.4f}, stale scales {stale:.4f} (torch BF16 product); "
+          f"vs oracle MXFP8 GEMM: healthy {e_ok:.2e}, stale {e_bad:.4f}; vs exact product: healthy {x_ok:.4f}, "
+          f"stale {x_bad:.4f}")
 
 
 def test_expert_probe_healthy_and_repacked_experts():
@@ -86,4 +124,19 @@ def test_expert_probe_healthy_and_repacked_experts():
     healthy = rel_err(mx.grouped_gemm(qx, sx, q, s, off), ref)
     repacked = rel_err(mx.grouped_gemm(qx, sx, q_bad, s_bad, off), ref)
     assert healthy < 0.1 and repacked > 1.0
-    print(f"expert probe: relative error healthy {healthy:.4f}, repacked experts {repacked:.4f}")
+
+    # Against the oracle: its grouped MXFP8 GEMM of the learner's grid, and the exact product.
+    qx_o, sx_o = oracle.quantize_rowwise(x.cpu())
+    qw_o, sw_o = oracle.quantize_rowwise(w.reshape(G * N, K).cpu())
+    ref_mx, _ = oracle.grouped_gemm(qx_o, sx_o, qw_o.reshape(G, N, K), sw_o.reshape(G, N, K // 32), o)
+    xs, ws = bf16_f64(x), bf16_f64(w)
+    exact = np.concatenate([xs[o[g]:o[g + 1]] @ ws[g].T for g in range(G)])
+    y_ok = to_np(mx.grouped_gemm(qx, sx, q, s, off).float())
+    y_bad = to_np(mx.grouped_gemm(qx, sx, q_bad, s_bad, off).float())
+    e_ok, e_bad = rel_err_np(y_ok, ref_mx), rel_err_np(y_bad, ref_mx)
+    x_ok, x_bad = rel_err_np(y_ok, exact), rel_err_np(y_bad, exact)
+    assert e_ok <= 2.0 ** -8 and e_bad > 1.0
+    assert x_ok < 0.1 and x_bad > 1.0
+    print(f"expert probe: relative error healthy {healthy:.4f}, repacked experts {repacked:.4f} (torch BF16 "
+          f"product); vs oracle MXFP8 GEMM: healthy {e_ok:.2e}, repacked {e_bad:.4f}; vs exact product: "
+          f"healthy {x_ok:.4f}, repacked {x_bad:.4f}")
