@@ -774,7 +774,9 @@ def run_library_gemm_peak(device, reps=10):
     return out
 
 
-BREAKEVEN_TOKENS = (1312, 2592, 5216, 10304)   # 1.3k / 2.6k / 5.2k / 10.3k rounded to multiples of 32
+# The pages' micro-batch sweep (Table 5: 1.3k / 2.6k / 5.2k / 10.3k tokens) rounded to multiples of
+# 32 (the columnwise copy of the wgrad operands needs it), plus 512 / 3.9k / 7.7k to pin the fit.
+BREAKEVEN_TOKENS = (512, 1312, 2592, 3904, 5216, 7744, 10304)
 BREAKEVEN_PASSES = 3
 
 
@@ -788,11 +790,17 @@ def fit_line(xs, ys):
 
 def breakeven_fit(points):
     """The pages' stage cost model t = delta + c * tokens fitted per path over one sweep, and the
-    break-even tokens per micro-batch m* = (delta_mxfp8 - delta_bf16) / (c_bf16 - c_mxfp8)."""
+    break-even tokens per micro-batch m* = (delta_mxfp8 - delta_bf16) / (c_bf16 - c_mxfp8). When the
+    points carry the paired difference "diff_ms" (MXFP8 - BF16, measured replay by replay), the
+    difference line is fitted directly: d = d_delta - d_c * tokens."""
     xs = [p["tokens"] for p in points]
     d_b, c_b = fit_line(xs, [p["bf16_ms"] for p in points])
     d_m, c_m = fit_line(xs, [p["mxfp8_ms"] for p in points])
-    dd, dc = d_m - d_b, c_b - c_m
+    if all("diff_ms" in p for p in points):
+        dd, neg_dc = fit_line(xs, [p["diff_ms"] for p in points])
+        dc = -neg_dc
+    else:
+        dd, dc = d_m - d_b, c_b - c_m
     return {"bf16": {"delta_ms": round(d_b, 4), "c_us_per_token": round(c_b * 1e3, 5)},
             "mxfp8": {"delta_ms": round(d_m, 4), "c_us_per_token": round(c_m * 1e3, 5)},
             "delta_delta_ms": round(dd, 4), "delta_c_us_per_token": round(dc * 1e3, 5),
@@ -803,23 +811,26 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
     """Kernel-level fixed cost and per-token cost of one update micro-batch of a Qwen3-8B linear
     (W 12288 x 4096, the TP-2 gate_up shard): BF16 (cuBLAS fprop, dgrad, wgrad) against MXFP8
     (quantize X and dY row+col with the scale layout, then the three MXFP8 GEMMs), each micro-batch
-    one CUDA graph, L2 flushed before each replay. The sweep over token counts is repeated `passes`
-    times, interleaved (every graph of a pass before the next pass), and the pages' stage cost
-    model t = delta + c * tokens (Table 7) is fitted per pass and path; m* = (delta_mxfp8 -
-    delta_bf16) / (c_bf16 - c_mxfp8) is reported per pass, with the fit of the per-point medians
-    and the spread. The weight's own quantization happens once per optimizer step, not per
-    micro-batch, and is reported beside the fit."""
+    one CUDA graph, L2 flushed before each replay. At each token count the two paths' replays
+    alternate one by one (the SM clock moves with the power cap, and pairing puts both paths under
+    the same conditions); the sweep is repeated `passes` times. Per pass the pages' stage cost model
+    t = delta + c * tokens (Table 7) is fitted to each path, and the paired difference MXFP8 - BF16
+    to a line d_delta - d_c * tokens, whose root m* = d_delta / d_c is the break-even tokens per
+    micro-batch; the result is the fit over all passes' per-point medians, with each pass's m*
+    beside it. The weight's own quantization happens once per optimizer step, not per micro-batch,
+    and is reported beside the fit."""
     import torch
 
     from mxfp8_block_scaled_07_b200 import mx, synth
 
     stream = torch.cuda.Stream(device)
+    cur = torch.cuda.current_stream()
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     O, H = 12288, 4096
     W = synth.normal_bf16((O, H), std=0.02, seed=61, device=device)
     qw = mx.quantize(W, True, True)
-    wq_ms = time_gpu(lambda: mx.quantize(W, True, True, out=qw), reps, flush, torch.cuda.current_stream())
-    graphs = []               # (tokens, path, graph), buffers kept alive in `keep`
+    wq_ms = time_gpu(lambda: mx.quantize(W, True, True, out=qw), reps, flush, cur)
+    graphs = {}               # tokens -> (bf16 graph, mxfp8 graph); buffers kept alive in `keep`
     keep = []
     for T in BREAKEVEN_TOKENS:
         X = synth.normal_bf16((T, H), std=1.0, seed=62, device=device)
@@ -843,30 +854,48 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
             mx.gemm(qd[0], qd[1], qw[2], qw[3], out=dX)
             mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW)
 
-        for name, fn in (("bf16", bf16_step), ("mxfp8", mxfp8_step)):
+        pair = []
+        for fn in (bf16_step, mxfp8_step):
             with torch.cuda.stream(stream):
                 fn()                                  # warm-up outside capture
             stream.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
-            graphs.append((T, name, g))
+            pair.append(g)
+        graphs[T] = pair
     torch.cuda.synchronize()
     mx.device_error()
+
+    def one(g):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        g.replay()
+        e1.record(cur)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+
     per_pass = []
     for _ in range(passes):
-        t = {}
-        for T, name, g in graphs:
-            t[(T, name)] = time_gpu(g.replay, reps, flush, torch.cuda.current_stream())
-        per_pass.append([{"tokens": T, "bf16_ms": round(t[(T, "bf16")], 4), "mxfp8_ms": round(t[(T, "mxfp8")], 4)}
-                         for T in BREAKEVEN_TOKENS])
+        pts = []
+        for T in BREAKEVEN_TOKENS:
+            gb, gm = graphs[T]
+            one(gb), one(gm)
+            tb, tm = [], []
+            for _ in range(reps):
+                tb.append(one(gb))
+                tm.append(one(gm))
+            pts.append({"tokens": T, "bf16_ms": round(statistics.median(tb), 4),
+                        "mxfp8_ms": round(statistics.median(tm), 4),
+                        "diff_ms": round(statistics.median(m - b for b, m in zip(tb, tm)), 4)})
+        per_pass.append(pts)
     status = device_status()
     del graphs, keep
     torch.cuda.synchronize()
     fits = [breakeven_fit(p) for p in per_pass]
-    med = [{"tokens": T,
-            "bf16_ms": round(statistics.median(p[i]["bf16_ms"] for p in per_pass), 4),
-            "mxfp8_ms": round(statistics.median(p[i]["mxfp8_ms"] for p in per_pass), 4)}
+    med = [{"tokens": T, **{k: round(statistics.median(p[i][k] for p in per_pass), 4)
+                            for k in ("bf16_ms", "mxfp8_ms", "diff_ms")}}
            for i, T in enumerate(BREAKEVEN_TOKENS)]
     out = {"linear": "W 12288x4096 (fprop, dgrad, wgrad per micro-batch)", "points": med, **breakeven_fit(med)}
     ms_ = [f["m_star_tokens"] for f in fits if f["m_star_tokens"] is not None]
@@ -876,8 +905,9 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
     if ms_:
         out["m_star_range"] = [min(ms_), max(ms_)]
     out["weight_quantize_row_col_ms_per_step"] = round(wq_ms, 4)
-    out["timing"] = (f"one CUDA graph per micro-batch and path; {passes} interleaved passes, median of {reps} "
-                     "replays per point and pass, L2 flushed before each; points = per-point medians over passes")
+    out["timing"] = (f"one CUDA graph per micro-batch and path; BF16 and MXFP8 replays alternated, {reps} pairs per "
+                     f"point and pass, {passes} passes, L2 flushed before each replay; m* from the paired "
+                     "difference line fitted to the per-point medians over passes")
     out.update(status)
     return out
 

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/mx.h"
 #include "blockwise.cuh"
@@ -182,18 +183,59 @@ EncodeTiledFn encode_fn() {
     return g_encode;
 }
 
+// Encoded 2-D tensor maps, cached per host thread. A map is a pure function of its arguments (base
+// address, sizes, stride, box, element type, swizzle), so a cached map is never stale; the cache only
+// saves the driver call (a few microseconds of host time per map) on repeated calls.
+struct TmapKey {
+    uintptr_t base;
+    uint64_t d0, d1, stride;
+    uint32_t b0, b1, kind;
+    bool operator==(const TmapKey& o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 && b1 == o.b1 &&
+               kind == o.kind;
+    }
+};
+struct TmapKeyHash {
+    size_t operator()(const TmapKey& k) const {
+        uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+        for (uint64_t v : {k.d0, k.d1, k.stride, uint64_t(k.b0) << 32 | k.b1, uint64_t(k.kind)})
+            h = (h ^ v) * 0x100000001B3ull;
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+constexpr size_t kTmapCacheMax = 4096;
+
+// kind: 0 = E4M3 operand (uint8, 128-byte swizzle), 1 = scale layout (uint8, no swizzle),
+// 2 = BF16 quantizer input (128-byte swizzle).
+bool encode_2d(CUtensorMap* map, uint32_t kind, const void* base, uint64_t d0, uint64_t d1, uint64_t stride,
+               uint32_t b0, uint32_t b1) {
+    static thread_local std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> cache;
+    const TmapKey key{reinterpret_cast<uintptr_t>(base), d0, d1, stride, b0, b1, kind};
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *map = it->second;
+        return true;
+    }
+    if (!encode_fn()) return false;
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {stride};
+    const cuuint32_t box[2] = {b0, b1};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = kind == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUtensorMapSwizzle sw = kind == 1 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    if (cache.size() >= kTmapCacheMax) cache.clear();
+    cache.emplace(key, *map);
+    return true;
+}
+
 // Tensor map of a K-major E4M3 operand [rows, cols_bytes]: boxes of box_rows x box_cols bytes with
 // the 128-byte swizzle the UMMA descriptors expect.
 bool make_tmap(CUtensorMap* map, const void* base, uint64_t cols_bytes, uint64_t rows, uint32_t box_cols,
                uint32_t box_rows) {
-    if (!encode_fn()) return false;
-    const cuuint64_t dims[2] = {cols_bytes, rows};
-    const cuuint64_t strides[1] = {cols_bytes};
-    const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(map, 0, base, cols_bytes, rows, cols_bytes, box_cols, box_rows);
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -225,14 +267,7 @@ int vector_store_ok(const void* c, int64_t ld_c, mx_out_dtype dt) {
 // bytes: one block is a 2-row box (loaded by the CTA-pair GEMM through TMA so that the peer CTA's
 // copies count on the leader's barrier).
 bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t blocks) {
-    if (!encode_fn()) return false;
-    const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(2 * blocks)};
-    const cuuint64_t strides[1] = {256};
-    const cuuint32_t box[2] = {256, 2};
-    const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(map, 1, base, 256, static_cast<uint64_t>(2 * blocks), 256, 256, 2);
 }
 
 // Launches the CTA-pair GEMM with a cluster dimension of 2.
@@ -362,14 +397,8 @@ mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceI
 // Tensor map of a BF16 input [M, K] (row stride ld_x elements) in 64-column x 128-row boxes with the
 // 128-byte swizzle the TMA-staged quantizer reads; out-of-range elements arrive as zeros.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t M, int64_t K, int64_t ld_x) {
-    if (!encode_fn()) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
-    const cuuint32_t box[2] = {64, 128};
-    const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(map, 2, base, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ld_x) * 2,
+                     64, 128);
 }
 
 template <int NT>

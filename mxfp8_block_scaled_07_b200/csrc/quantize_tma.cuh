@@ -97,10 +97,27 @@ __device__ __forceinline__ QtTile qt_decode(const QuantTmaArgs<NT>& a, int64_t t
     return r;
 }
 
-// Requests tile t into stage buffer `dst` (one thread): one box per 64-column half that overlaps K.
+// The tile after r in the launch's tile space (row-major within a tensor, tensors in order).
 template <int NT>
-__device__ __forceinline__ void qt_issue(const QuantTmaArgs<NT>& a, int64_t t, uint32_t dst, uint64_t* bar) {
-    const QtTile r = qt_decode(a, t);
+__device__ __forceinline__ void qt_next(const QuantTmaArgs<NT>& a, QtTile& r) {
+    if (++r.kt == a.t[r.i].tiles_k) {
+        r.kt = 0;
+        if (++r.mt == a.t[r.i].tiles_m) {
+            r.mt = 0;
+            ++r.i;
+        }
+    }
+    if (r.i < a.n) {
+        const QtTensor& T = a.t[r.i];
+        r.m0 = static_cast<int64_t>(r.mt) * kQTile;
+        r.k0 = static_cast<int64_t>(r.kt) * kQTile;
+        r.full = (r.m0 + kQTile <= T.M) && (r.k0 + kQTile <= T.K);
+    }
+}
+
+// Requests tile r into stage buffer `dst` (one thread): one box per 64-column half that overlaps K.
+template <int NT>
+__device__ __forceinline__ void qt_issue(const QuantTmaArgs<NT>& a, const QtTile& r, uint32_t dst, uint64_t* bar) {
     const bool second = r.k0 + 64 < a.t[r.i].K;
     mbar_arrive_expect_tx(bar, second ? kQtStageBytes : kQtHalfBytes);
     const uint32_t b = smem_u32(bar);
@@ -133,16 +150,21 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tma_kernel(const __grid
         fence_barrier_init();
     }
     __syncthreads();
+    // Tiles are walked incrementally: every thread steps `rc` through its CTA's range, and thread 0
+    // also steps `ri`, the next tile to request (kQtStages ahead).
+    QtTile rc, ri;
+    if (t_begin < t_end) rc = ri = qt_decode(a, t_begin);
     if (tid == 0)
-        for (int s = 0; s < kQtStages && t_begin + s < t_end; ++s)
-            qt_issue(a, t_begin + s, stages_s + s * kQtStageBytes, &full[s]);
+        for (int s = 0; s < kQtStages && t_begin + s < t_end; ++s) {
+            qt_issue(a, ri, stages_s + s * kQtStageBytes, &full[s]);
+            qt_next(a, ri);
+        }
 
     int64_t t = t_begin;
-    for (int j = 0; t < t_end; ++t, ++j) {
+    for (int j = 0; t < t_end; ++t, ++j, qt_next(a, rc)) {
         const int s = j % kQtStages;
         const bool ok = mbar_wait(&full[s], static_cast<uint32_t>(j / kQtStages) & 1u, abort, a.err, a.timeout_ns);
         if (__syncthreads_or(!ok)) break;
-        const QtTile rc = qt_decode(a, t);
         const QtTensor& T = a.t[rc.i];
         const uint32_t st = stages_s + s * kQtStageBytes;
         uint8_t* atom_row = atoms + (j & 1) * 1024;
@@ -226,7 +248,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tma_kernel(const __grid
             }
         }
         __syncthreads();     // stage s read by every thread; this tile's scale blocks complete
-        if (tid == 0 && t + kQtStages < t_end) qt_issue(a, t + kQtStages, st, &full[s]);
+        if (tid == 0 && t + kQtStages < t_end) {
+            qt_issue(a, ri, st, &full[s]);
+            qt_next(a, ri);
+        }
         // Scale output: one 512-byte block of the tensor-core layout per direction, or raw bytes. The
         // other pair of atom buffers takes the next tile, so no second barrier is needed here.
         if constexpr (ROW) {

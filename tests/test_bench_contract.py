@@ -48,3 +48,19 @@ def test_breakeven_fit_recovers_the_stage_cost_model():
     # No saving per token: no break-even.
     flat = [{"tokens": T, "bf16_ms": 1.0, "mxfp8_ms": 2.0} for T in bench.BREAKEVEN_TOKENS]
     assert bench.breakeven_fit(flat)["m_star_tokens"] is None
+
+
+def test_breakeven_fit_from_paired_differences():
+    """With paired differences the difference line is fitted directly; on exact data it agrees with
+    the two per-path fits."""
+    import pytest
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    pts = [{"tokens": T, "bf16_ms": 0.020 + 2.0e-4 * T, "mxfp8_ms": 0.030 + 1.3e-4 * T,
+            "diff_ms": 0.010 - 7.0e-5 * T} for T in bench.BREAKEVEN_TOKENS]
+    f = bench.breakeven_fit(pts)
+    assert f["delta_delta_ms"] == pytest.approx(0.010, abs=1e-4)
+    assert f["delta_c_us_per_token"] == pytest.approx(0.07, rel=1e-3)
+    assert f["m_star_tokens"] == pytest.approx(0.010 / 7.0e-5, rel=1e-3)
