@@ -810,8 +810,8 @@ def breakeven_fit(points):
 def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
     """Kernel-level fixed cost and per-token cost of one update micro-batch of a Qwen3-8B linear
     (W 12288 x 4096, the TP-2 gate_up shard): BF16 (cuBLAS fprop, dgrad, wgrad) against MXFP8
-    (quantize X and dY row+col with the scale layout, then the three MXFP8 GEMMs), each micro-batch
-    one CUDA graph, L2 flushed before each replay. At each token count the two paths' replays
+    (X and dY quantized row+col with the scale layout in one multi-tensor launch, then the three
+    MXFP8 GEMMs), each micro-batch one CUDA graph, L2 flushed before each replay. At each token count the two paths' replays
     alternate one by one (the SM clock moves with the power cap, and pairing puts both paths under
     the same conditions); the sweep is repeated `passes` times. Per pass the pages' stage cost model
     t = delta + c * tokens (Table 7) is fitted to each path, and the paired difference MXFP8 - BF16
@@ -848,8 +848,7 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
             torch.matmul(dY.t(), X, out=dW)
 
         def mxfp8_step(X=X, dY=dY, Y=Y, dX=dX, dW=dW, qx=qx, qd=qd):
-            mx.quantize(X, True, True, out=qx)
-            mx.quantize(dY, True, True, out=qd)
+            mx.quantize_multi([X, dY], True, True, swizzle=True, outs=[qx, qd])   # one launch for both
             mx.gemm(qx[0], qx[1], qw[0], qw[1], out=Y)
             mx.gemm(qd[0], qd[1], qw[2], qw[3], out=dX)
             mx.gemm(qd[2], qd[3], qx[2], qx[3], out=dW)

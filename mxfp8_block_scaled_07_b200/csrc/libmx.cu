@@ -79,7 +79,7 @@ int max_pair_clusters(K kernel, int smem, int sms) {
 
 // GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
 std::atomic<int> g_gemm_variant{0};
-// Quantizer selection: 0 = TMA-staged tiles (default), 1 = register-staged tiles.
+// Quantizer selection: 0 = register-staged tiles (default), 1 = TMA-staged tiles.
 std::atomic<int> g_quant_variant{0};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -473,7 +473,7 @@ mx_status mx_quantize(const void* x, int64_t M, int64_t K, int64_t ld_x, int fla
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    if (g_quant_variant.load() == 0) {
+    if (g_quant_variant.load() == 1) {
         QuantTmaArgs<1> a;
         a.n = 0;
         a.swz = swz;
@@ -503,7 +503,7 @@ mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags
     if (n == 0) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    if (g_quant_variant.load() == 0) {
+    if (g_quant_variant.load() == 1) {
         static thread_local QuantTmaArgs<kQtMaxTensors> a;   // ~30 KB: kept off the stack
         for (int64_t i0 = 0; i0 < n; i0 += kQtMaxTensors) {
             a.n = 0;

@@ -334,6 +334,19 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t saddr) {
     return v;
 }
 
+// Largest magnitude bits of each half over w[0..31] (two columns of a 32-row block), as a tree of
+// depth 5 rather than a chain of 32 dependent maxima.
+__device__ __forceinline__ uint32_t col_pair_absmax(const uint32_t (&w)[32]) {
+    uint32_t m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m[i] = bf16x2_absmax(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+    for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+        for (int i = 0; i < n; ++i) m[i] = bf16x2_absmax(m[i], m[i + n]);
+    return m[0] & 0x7FFF7FFFu;
+}
+
 // The 32 BF16 of one column (the low or the high halves of w[0..31]) -> 32 E4M3 bytes, row i in
 // byte i of the result.
 __device__ __forceinline__ void encode_col32(const uint32_t (&w)[32], uint32_t s, bool hi, uint32_t (&o)[8]) {
@@ -444,10 +457,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 w[i] = ld_shared_u32(tile_s + qtile_chunk(mb * 32 + i, cp >> 2) + (cp & 3) * 4);
-            uint32_t m = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) m = bf16x2_absmax(m, w[i]);
-            m &= 0x7FFF7FFFu;
+            const uint32_t m = col_pair_absmax(w);
             const int64_t kc = rc.k0 + 2 * cp;           // K-row of the transposed copy (low halves)
             const int64_t mr = rc.m0 + 32 * mb;
             const bool mok = rc.full || mr < T.M;        // M % 32 == 0: a block is all in or all out

@@ -219,10 +219,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tma_kernel(const __grid
             uint32_t w[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) w[i] = ld_shared_u32(base + qt_chunk(mb * 32 + i, cc));
-            uint32_t m = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) m = bf16x2_absmax(m, w[i]);
-            m &= 0x7FFF7FFFu;
+            const uint32_t m = col_pair_absmax(w);
             const int64_t kc = rc.k0 + 2 * cp;           // K-row of the transposed copy (low halves)
             const int64_t mr = rc.m0 + 32 * mb;
             const bool mok = rc.full || mr < T.M;        // M % 32 == 0: a block is all in or all out

@@ -303,9 +303,9 @@ def set_gemm_variant(variant: int):
     lib().mx_set_gemm_variant(int(variant))
 
 
-QUANT_TMA, QUANT_REGISTERS = 0, 1
+QUANT_REGISTERS, QUANT_TMA = 0, 1
 
 
 def set_quantize_variant(variant: int):
-    """0: TMA-staged quantizer (default); 1: register-staged quantizer. Same bytes either way."""
+    """0: register-staged quantizer (default); 1: TMA-staged quantizer. Same bytes either way."""
     lib().mx_set_quantize_variant(int(variant))

@@ -39,9 +39,9 @@ def gemm_variant(request):
     mx.set_gemm_variant(0)
 
 
-@pytest.fixture(params=[0, 1], ids=["tma", "regs"])
+@pytest.fixture(params=[0, 1], ids=["regs", "tma"])
 def quant_variant(request):
-    """Runs a quantizer test with the TMA-staged kernel (0, the default) and the register-staged
+    """Runs a quantizer test with the register-staged kernel (0, the default) and the TMA-staged
     kernel (1)."""
     from mxfp8_block_scaled_07_b200 import mx
 
