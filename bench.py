@@ -994,6 +994,8 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1],
                     help="GEMM kernel for --case runs: 0 CTA pair (default), 1 single CTA")
+    ap.add_argument("--quant-variant", type=int, default=0, choices=[0, 1],
+                    help="quantizer kernel for --case runs: 0 register-staged (default), 1 TMA-staged")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -1008,6 +1010,7 @@ def main():
 
         mxbuild.build()
         mx.set_gemm_variant(args.gemm_variant)
+        mx.set_quantize_variant(args.quant_variant)
         return run_case(args.case, args.reps)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

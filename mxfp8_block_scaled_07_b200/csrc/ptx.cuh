@@ -197,9 +197,14 @@ __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr)
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
     return v;
 }
-// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA), with the
+// default CTA-scope release. The GEMM epilogue arrives this way to hand accumulator columns back to
+// the MMA issuer; what must be ordered before the arrive are its TMEM loads, which tcgen05.wait::ld
+// completes and tcgen05.fence::before_thread_sync orders. A cluster-scope release would also wait
+// until the warp's earlier global stores of C are acknowledged, about 6k cycles per tile on the
+// B200; the MMA issuer never reads C.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),
