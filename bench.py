@@ -514,7 +514,13 @@ def aggregate_e2e(pg, local: dict, world: int, bytes_per_rank_step: int, device=
 
 
 def flush_l2(buf):
-    buf.add_(1)
+    """Evicts the timed kernel's data from L2 before a timed launch: writes a buffer larger than L2,
+    then reads a second one, so that the written lines are written back here and not during the
+    timed launch (a flush that only writes leaves up to 126 MB of dirty lines that the next kernel
+    pays to write back). `buf` holds both halves."""
+    h = buf.numel() // 2
+    buf[:h].add_(1)
+    buf[h:].sum()
 
 
 def time_gpu(fn, reps, flush_buf, stream):
@@ -584,7 +590,7 @@ def run_secondary(device, peaks, reps=10):
     from mxfp8_block_scaled_07_b200 import mx, synth
 
     stream = torch.cuda.current_stream()
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    flush = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=device)   # 2 x (2 x L2)
     fp8_peak = peaks["bf16_tflops"] * NOMINAL_FP8_OVER_BF16
     out = {"gemm": [], "quantize": [], "fp8_peak_tflops": round(fp8_peak, 1),
            "fp8_peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
@@ -744,7 +750,7 @@ def run_library_gemm_peak(device, reps=10):
 
     n = 8192
     stream = torch.cuda.current_stream()
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    flush = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=device)   # 2 x (2 x L2)
     A = synth.normal_bf16((n, n), std=1.0, seed=51, device=device)
     B = synth.normal_bf16((n, n), std=1.0, seed=52, device=device)
     qa, sa, _, _ = mx.quantize(A, True, False)
@@ -825,7 +831,7 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
 
     stream = torch.cuda.Stream(device)
     cur = torch.cuda.current_stream()
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    flush = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=device)   # 2 x (2 x L2)
     O, H = 12288, 4096
     W = synth.normal_bf16((O, H), std=0.02, seed=61, device=device)
     qw = mx.quantize(W, True, True)

@@ -216,10 +216,11 @@ void mx_set_gemm_variant(int variant);
 /*
  * Selects the quantizer kernel behind later mx_quantize / mx_quantize_multi calls (process-wide):
  * 0 (default) loads each thread's two 32-element blocks of a 128 x 128 BF16 tile into registers
- * with 256-bit loads, one tile ahead of the compute (the columnwise pass goes through a swizzled
- * shared-memory copy of the tile); 1 stages the tiles in shared memory with TMA tensor loads
- * running three tiles ahead. Both produce the same bytes; 0 measured faster on B200 (see the
- * design notes). Other values select 0.
+ * with 256-bit loads, one tile ahead of the compute (the columnwise pass of a row + col call goes
+ * through a swizzled shared-memory copy of the tile), except that columnwise-only calls take the
+ * TMA-staged kernel; 1 stages the tiles of every call in shared memory with TMA tensor loads
+ * running three tiles ahead. Both produce the same bytes; the default picks the kernel measured
+ * faster on B200 for each direction. Other values select 0.
  */
 void mx_set_quantize_variant(int variant);
 

@@ -79,8 +79,11 @@ int max_pair_clusters(K kernel, int smem, int sms) {
 
 // GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
 std::atomic<int> g_gemm_variant{0};
-// Quantizer selection: 0 = register-staged tiles (default), 1 = TMA-staged tiles.
+// Quantizer selection: 0 = register-staged tiles (default; columnwise-only calls take the TMA-staged
+// kernel, measured faster for that direction), 1 = TMA-staged tiles.
 std::atomic<int> g_quant_variant{0};
+
+bool use_tma_quantizer(bool row, bool col) { return g_quant_variant.load() == 1 || (col && !row); }
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -133,7 +136,6 @@ const DeviceInfo* device_info() {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1], quantize_rowwise_kernel<kQMaxTensors>,
                                                       kQThreads, 0);
         if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
-        d.quant_blocks_per_sm[2] = quant_occupancy<false>();
         d.quant_blocks_per_sm[3] = quant_occupancy<true>();
         if (!qt_setup<true, false>(&d.qt_blocks_per_sm[1]) || !qt_setup<false, true>(&d.qt_blocks_per_sm[2]) ||
             !qt_setup<true, true>(&d.qt_blocks_per_sm[3]))
@@ -385,12 +387,10 @@ mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceI
     if (a.total_tiles == 0) return MX_OK;
     const int which = (row ? 1 : 0) | (col ? 2 : 0);
     const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
-    if (row && col)
+    if (col)     // row + col (columnwise only takes the TMA-staged kernel)
         quantize_rowcol_kernel<true, NT><<<grid, kQThreads, 0, stream>>>(a);
-    else if (row)
-        quantize_rowwise_kernel<NT><<<grid, kQThreads, 0, stream>>>(a);
     else
-        quantize_rowcol_kernel<false, NT><<<grid, kQThreads, 0, stream>>>(a);
+        quantize_rowwise_kernel<NT><<<grid, kQThreads, 0, stream>>>(a);
     return launched();
 }
 
@@ -473,7 +473,7 @@ mx_status mx_quantize(const void* x, int64_t M, int64_t K, int64_t ld_x, int fla
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    if (g_quant_variant.load() == 1) {
+    if (use_tma_quantizer(row, col)) {
         QuantTmaArgs<1> a;
         a.n = 0;
         a.swz = swz;
@@ -503,7 +503,7 @@ mx_status mx_quantize_multi(const mx_quant_tensor* tensors, int64_t n, int flags
     if (n == 0) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    if (g_quant_variant.load() == 1) {
+    if (use_tma_quantizer(row, col)) {
         static thread_local QuantTmaArgs<kQtMaxTensors> a;   // ~30 KB: kept off the stack
         for (int64_t i0 = 0; i0 < n; i0 += kQtMaxTensors) {
             a.n = 0;

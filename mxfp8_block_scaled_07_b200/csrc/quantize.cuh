@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
     }
 }
 
-// ---- rowwise + columnwise (or columnwise only) kernel --------------------------------------
+// ---- rowwise + columnwise kernel -------------------------------------------------------------
 //
 // Same tile walk and block-per-thread rowwise pass as above. Each thread also stages its two
 // BF16 blocks in shared memory (128 rows x 256 bytes; 16-byte chunks XOR-swizzled so that both
