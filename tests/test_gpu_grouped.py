@@ -52,7 +52,7 @@ def grouped_case(counts, N, K, out_dtype, seed=0, device_inputs=None):
 
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_grouped_small_ragged_with_empty_groups(out_dtype, gemm_variant):
+def test_grouped_small_ragged_with_empty_groups(out_dtype, grouped_variant):
     counts = [0, 5, 128, 129, 300, 0, 1, 64, 256, 257, 511, 2]
     N, K = 384, 256
     X, W, off, c = grouped_case(counts, N, K, out_dtype, seed=3)
@@ -62,7 +62,7 @@ def test_grouped_small_ragged_with_empty_groups(out_dtype, gemm_variant):
     assert_gemm_close(to_np(c.float()), ref, abs_sum, out_dtype == torch.bfloat16, "grouped small")
 
 
-def test_grouped_bad_offsets_set_device_error_and_write_nothing(gemm_variant):
+def test_grouped_bad_offsets_set_device_error_and_write_nothing(grouped_variant):
     counts = [64, 64]
     N, K = 256, 128
     X = synth.normal_bf16((128, K), seed=1).cuda()
@@ -99,3 +99,31 @@ def test_moe_layer_full_size_sampled():
             ref, abs_sum = oracle.gemm(qa, sa, qb, sb)
             assert_gemm_close(to_np(c[torch.from_numpy(rr).cuda()][:, torch.from_numpy(cols).cuda()].float()),
                               ref, abs_sum, True, f"{name} expert {e}")
+
+
+@pytest.mark.parametrize("K", [32, 128, 384, 768, 896])
+@pytest.mark.parametrize("N", [128, 200, 640])
+def test_grouped_short_k_shapes(K, N, grouped_variant):
+    """Around the resident-A kernel's range (K <= 768: 1..6 resident k-blocks; 896 falls back to the
+    pair kernel) with N not a multiple of 128 and experts of 0, 1, 128, 255, 256 and 300 rows."""
+    counts = [128, 0, 1, 300, 255, 256, 3]
+    X, W, off, c = grouped_case(counts, N, K, torch.float32, seed=K + N)
+    qx, sx = oracle.quantize_rowwise(X)
+    qw, sw = oracle.quantize_rowwise(W.reshape(-1, K))
+    G = len(counts)
+    ref, abs_sum = oracle.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw.reshape(G, N, K // 32), off)
+    assert_gemm_close(to_np(c), ref, abs_sum, False, f"grouped K={K} N={N}")
+
+
+def test_grouped_many_units_per_pair():
+    """More m-tiles than CTA pairs (each pair walks several units, so resident A slots are refilled
+    while B of the previous unit is still in flight), 40 experts of up to 700 rows, K = 768."""
+    g = np.random.default_rng(11)
+    counts = [int(c) for c in g.integers(0, 700, 40)]
+    N, K = 384, 768
+    X, W, off, c = grouped_case(counts, N, K, torch.bfloat16, seed=5)
+    qx, sx = oracle.quantize_rowwise(X)
+    qw, sw = oracle.quantize_rowwise(W.reshape(-1, K))
+    G = len(counts)
+    ref, abs_sum = oracle.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw.reshape(G, N, K // 32), off)
+    assert_gemm_close(to_np(c.float()), ref, abs_sum, True, "grouped many units")
