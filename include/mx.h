@@ -206,14 +206,10 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
                                float* scales, mx_stream stream);
 
 /*
- * Selects the kernel behind later mx_gemm / mx_grouped_gemm calls (process-wide):
- *   0 (default): CTA-pair kernels (two SMs per tile with tcgen05.mma.cta_group::2): 256 x 256 tiles,
- *                except mx_grouped_gemm with K <= 768, which keeps each expert's 256-row A tile
- *                resident in shared memory and computes 256 x 128 tiles;
- *   1: the single-CTA kernel (128 x 256 tiles);
- *   2: the 256 x 256 CTA-pair kernel for every shape.
- * All meet the accuracy bound above; results may differ in fp32 summation order only. Other values
- * select 0.
+ * Selects the kernel behind later mx_gemm / mx_grouped_gemm calls (process-wide): 0 (default) the
+ * CTA-pair kernel (256 x 256 tiles computed by two SMs with tcgen05.mma.cta_group::2), 1 the
+ * single-CTA kernel (128 x 256 tiles). Both meet the accuracy bound above; results may differ in
+ * fp32 summation order only. Other values select 0.
  */
 void mx_set_gemm_variant(int variant);
 

@@ -204,28 +204,22 @@ __device__ __forceinline__ Tile decode_tile_pair(int t, int rank, const GemmArgs
 // 4 rows per instruction), masked to the tile's valid rows and to N. The stores go through the
 // load/store path, not TMA: TMA stores share the SM's TMA unit with the operand loads and were
 // measured to slow those down. Barrier addresses are shared::cluster addresses.
-// NCOL = 256 with OVL: the two overlapping 256-column accumulators (acc1 selects the second, whose
-// first 16 columns are the first's last 16). NCOL = 128 without OVL: a 128-column accumulator at
-// TMEM column acc_col, no shared columns (ovl_free_addr unused).
-template <bool GROUPED, int NCOL = 256, bool OVL = true>
+template <bool GROUPED>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, uint32_t tmem_base, bool acc1,
                                               uint8_t* stage, uint32_t ovl_free_addr, uint32_t acc_empty_addr,
-                                              int q, int lane, uint32_t acc_col = 0) {
-    static_assert((NCOL == 256 && OVL) || (NCOL == 128 && !OVL), "epilogue shapes");
+                                              int q, int lane) {
     const int warp_rows = min(32, max(0, T.rows_valid - q * 32));
     const int64_t row0 = static_cast<int64_t>(T.a_row0) + q * 32;
     const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t tq = lanes + (OVL ? (acc1 ? kAcc1Col : 0u) : acc_col);
+    const uint32_t tq = lanes + (acc1 ? kAcc1Col : 0u);
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
 
     uint32_t ov[16];                     // tile columns 240..255 of accumulator 0, 0..15 of accumulator 1
-    if constexpr (OVL) {
-        tc_ld_32x32b_x16(lanes + kOvlCol, ov);
-        tc_wait_ld_regs(ov);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
-    }
+    tc_ld_32x32b_x16(lanes + kOvlCol, ov);
+    tc_wait_ld_regs(ov);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(ovl_free_addr);
 
     // Writes one 128-byte row piece p (64 BF16 or 32 fp32 columns starting at col0) of the 32 rows.
     const uint32_t box = smem_u32(stage);
@@ -271,11 +265,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
     // Issues the TMEM loads of tile columns [32 c, 32 c + 32) into p; the shared columns come from `ov`.
     // The caller waits (tc_wait_ld_regs) before reading p.
     auto load32 = [&](int c, uint32_t(&p)[32]) {
-        if (OVL && acc1 && c == 0) {
+        if (acc1 && c == 0) {
             tc_ld_32x32b_x16(tq + 16u, *reinterpret_cast<uint32_t(*)[16]>(&p[16]));
 #pragma unroll
             for (int i = 0; i < 16; ++i) p[i] = ov[i];
-        } else if (OVL && !acc1 && c == 7) {
+        } else if (!acc1 && c == 7) {
             tc_ld_32x32b_x16(tq + 224u, *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
 #pragma unroll
             for (int i = 0; i < 16; ++i) p[16 + i] = ov[i];
@@ -295,10 +289,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
             pk[i] = *reinterpret_cast<const uint32_t*>(&v);
         }
     };
-    constexpr int kPieces = NCOL / 64;       // BF16: 64-column pieces
-    constexpr int kChunks = NCOL / 32;       // fp32: 32-column pieces
     if (a.out_bf16) {
-        // 64-column pieces; the next piece's TMEM loads are in flight while the current one is
+        // Four 64-column pieces; the next piece's TMEM loads are in flight while the current one is
         // stored, and the accumulator is released as soon as the last piece is in registers.
         uint32_t raw[64], pa[32], pb[32];
         load32(0, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
@@ -306,17 +298,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
         tc_wait_ld_regs(raw);
         pack(raw, pa);
 #pragma unroll
-        for (int ch = 0; ch < kPieces; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {
             uint32_t(&cur)[32] = (ch & 1) ? pb : pa;
             uint32_t(&nxt)[32] = (ch & 1) ? pa : pb;
-            if (ch < kPieces - 1) {
+            if (ch < 3) {
                 load32(2 * ch + 2, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
                 load32(2 * ch + 3, *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
             }
             emit(cur, T.n0 + ch * 64);
-            if (ch < kPieces - 1) {
+            if (ch < 3) {
                 tc_wait_ld_regs(raw);
-                if (ch == kPieces - 2) release();
+                if (ch == 2) release();
                 pack(raw, nxt);
             }
         }
@@ -326,14 +318,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& T, 
         load32(0, f0);
         tc_wait_ld_regs(f0);
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
+        for (int c = 0; c < 8; ++c) {
             uint32_t(&cur)[32] = (c & 1) ? f1 : f0;
             uint32_t(&nxt)[32] = (c & 1) ? f0 : f1;
-            if (c < kChunks - 1) load32(c + 1, nxt);
+            if (c < 7) load32(c + 1, nxt);
             emit(cur, T.n0 + c * 32);
-            if (c < kChunks - 1) {
+            if (c < 7) {
                 tc_wait_ld_regs(nxt);
-                if (c == kChunks - 2) release();
+                if (c == 6) release();
             }
         }
     }
@@ -816,301 +808,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             else if (i >= peer)
                 mbar_complete_tx(bar, kPairStageBytes);         // the peer never requested its half
             mbar_wait_drain(bar, (i / S) & 1u, a.timeout_ns);
-        }
-    }
-    cluster_sync();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem_base, kTmemCols);
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
-// Grouped CTA-pair kernel for short K (K <= 768, the MoE down projection): resident A.
-//
-// A unit is one 256-row m-tile of one expert (128 rows per CTA) with all its n-tiles of 128
-// columns. The unit's A tile (K / 128 <= 6 k-blocks of 16 KB per CTA, with their scale blocks) is
-// loaded once into resident slots and stays in shared memory while B streams through a 9-stage
-// ring of 8 KB (64 rows per CTA) stages. Per k-block of output this moves B plus a sixteenth of A
-// from L2 instead of both. Three 128-column TMEM accumulators ([0, 128), [128, 256), [256, 384))
-// plus one scale slot (SFA at 384, SFB at 388) fit without overlap, so a tile's MMAs never wait
-// for the previous tile's columns to be read out; the epilogue groups alternate tiles as in the
-// pair kernel. A resident slot is refilled for the next unit as soon as the MMAs of the unit's
-// last n-tile that read it have completed (a_empty, committed per slot), interleaved with the
-// next unit's first B stages. Units are dealt to the pairs round-robin, so the pairs in flight
-// work on neighbouring m-tiles and share B in L2. Same bounded waits, drain and error bits as the
-// pair kernel.
-// ---------------------------------------------------------------------------------------------
-constexpr int kAresMaxKb = 6;                          // K <= 6 * 128
-constexpr int kAresBN = 128;                           // output columns per tile
-constexpr int kAresStages = 9;                         // B ring
-constexpr uint32_t kAresAccCols = 128;
-constexpr uint32_t kAresSfCol = 3 * kAresAccCols;      // SFA [384, 388), SFB [388, 392)
-constexpr uint32_t kAresABytes = kBM * kBK + kSfaBytes;                 // per CTA and k-block
-constexpr uint32_t kAresBBytes = (kAresBN / 2) * kBK + kSfaBytes;       // per CTA and B stage
-
-struct AresSmem {
-    static constexpr int kA = 0;                                          // resident A slots
-    static constexpr int kSfa = kA + kAresMaxKb * kBM * kBK;
-    static constexpr int kB = kSfa + kAresMaxKb * kSfaBytes;              // B ring
-    static constexpr int kSfb = kB + kAresStages * (kAresBN / 2) * kBK;
-    static constexpr int kStage = (kSfb + kAresStages * kSfaBytes + 1023) / 1024 * 1024;
-    static constexpr int kBar = kStage + kEpiWarps * kStageBytes;
-    static constexpr int kNumBars = 2 * kAresMaxKb + 2 * kAresStages + 7;
-    static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kGroups = (kMisc + 32 + 15) / 16 * 16;
-    static constexpr int kBytes = kGroups + 3 * (kMaxGroups + 1) * 4 + 1024;   // + alignment slack
-};
-static_assert(AresSmem::kB % 1024 == 0 && AresSmem::kA % 1024 == 0, "swizzled operand buffers 1024-aligned");
-static_assert(AresSmem::kBytes <= 232448, "shared memory per CTA");
-constexpr int kGemmAresSmem = AresSmem::kBytes;
-
-struct AresUnit {
-    int a_row0;         // first A (and C) row of this CTA
-    int rows_valid;     // rows of C this CTA owns in the unit (0..128)
-    int sfa_tile;       // 128-row tile index into A's scale layout
-    int g;              // expert
-};
-
-__device__ __forceinline__ AresUnit decode_unit(int u, int rank, const GemmArgs& a, const int32_t* off,
-                                                const int32_t* pm128, const int32_t* pm256) {
-    AresUnit U;
-    U.g = find_group(pm256, a.G, u);
-    const int local = u - pm256[U.g];
-    U.a_row0 = off[U.g] + local * 2 * kBM + rank * kBM;
-    U.rows_valid = max(0, min(kBM, off[U.g + 1] - U.a_row0));
-    U.sfa_tile = min(pm128[U.g] + 2 * local + rank, pm128[a.G] - 1);
-    return U;
-}
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    mx_gemm_ares_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                        const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                        const GemmArgs a) {
-    using L = AresSmem;
-    constexpr int S = kAresStages;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // [6], leader: both CTAs' A slot landed
-    uint64_t* a_empty = a_full + kAresMaxKb;                          // [6]: the unit's MMAs on slot kb done
-    uint64_t* b_full = a_empty + kAresMaxKb;                          // [S], leader
-    uint64_t* b_empty = b_full + S;                                   // [S]
-    uint64_t* tmem_full = b_empty + S;                                // [3]: accumulator holds a finished tile
-    uint64_t* acc_empty = tmem_full + 3;                              // [3], leader: read out in both CTAs
-    uint64_t* drain = acc_empty + 3;
-    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-    uint32_t* b_issued_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc + 8);   // B stage fills
-    uint32_t* a_units_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc + 12);  // units whose A loads began
-    uint32_t* a_kb_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc + 16);     // A slots filled for the last
-    int32_t* off = reinterpret_cast<int32_t*>(smem + L::kGroups);
-    int32_t* pm128 = off + (kMaxGroups + 1);
-    int32_t* pm256 = pm128 + (kMaxGroups + 1);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int rank = static_cast<int>(cluster_ctarank());
-    const bool leader = rank == 0;
-    const int pair = blockIdx.x >> 1;
-    const int npairs = gridDim.x >> 1;
-
-    if (threadIdx.x == 0) {
-        for (int k = 0; k < kAresMaxKb; ++k) {
-            mbar_init(&a_full[k], 1);
-            mbar_init(&a_empty[k], 1);
-        }
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&b_full[s], 1);
-            mbar_init(&b_empty[s], 1);
-        }
-        for (int c = 0; c < 3; ++c) {
-            mbar_init(&tmem_full[c], 1);
-            mbar_init(&acc_empty[c], kEpiWarps);     // one arrive per warp of one group in both CTAs
-        }
-        mbar_init(drain, 1);
-        *abort = 0;
-        *b_issued_slot = 0;
-        *a_units_slot = 0;
-        *a_kb_slot = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmap_a);
-        prefetch_tensormap(&tmap_b);
-        prefetch_tensormap(&tmap_sfa);
-        prefetch_tensormap(&tmap_sfb);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(tmem_base_slot, kTmemCols);
-        tmem_relinquish_pair();
-    }
-    // Units: the groups' 256-row m-tiles (the tile count setup_groups returns for one n-tile column).
-    const int units = setup_groups(a, off, pm128, pm256, 1);
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();                         // both CTAs' barriers initialized before any remote signal
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_base_slot;
-    const int tiles_n = a.tiles_n;
-
-    if (warp == 0) {
-        // ---------------- TMA producer (both CTAs; completions counted in the leader) ----------------
-        int stage = 0;
-        uint32_t phase = 0, b_issued = 0, a_units = 0, a_kb = 0;
-        bool ok = true;
-        int ul = 0;
-        for (int u = pair; u < units && ok; u += npairs, ++ul) {
-            const AresUnit U = decode_unit(u, rank, a, off, pm128, pm256);
-            for (int i = 0; i < tiles_n && ok; ++i) {
-                const int b_row0 = U.g * a.N + i * kAresBN + rank * (kAresBN / 2);
-                const int sfb_tile = U.g * a.n_rowtiles + i;
-                for (int kb = 0; kb < a.nkb; ++kb) {
-                    if (i == 0) {   // refill resident slot kb once the previous unit is done with it
-                        if (ul > 0 && !mbar_wait(&a_empty[kb], static_cast<uint32_t>(ul - 1) & 1u, abort, a.err,
-                                                 a.timeout_ns)) {
-                            ok = false;
-                            break;
-                        }
-                        __syncwarp();
-                        const uint32_t fa = mapa_shared(smem_u32(&a_full[kb]), 0);
-                        if (leader) mbar_arrive_expect_tx_elect(&a_full[kb], 2 * kAresABytes);
-                        tma_load_2d_pair_elect(smem + L::kA + kb * kBM * kBK, &tmap_a, fa, kb * kBK, U.a_row0);
-                        tma_load_2d_pair_elect(smem + L::kSfa + kb * kSfaBytes, &tmap_sfa, fa, 0,
-                                               2 * (U.sfa_tile * a.nkb + kb));
-                        a_units = static_cast<uint32_t>(ul) + 1;
-                        a_kb = static_cast<uint32_t>(kb) + 1;
-                    }
-                    if (!mbar_wait(&b_empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
-                    __syncwarp();
-                    const uint32_t fb = mapa_shared(smem_u32(&b_full[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx_elect(&b_full[stage], 2 * kAresBBytes);
-                    tma_load_2d_pair_elect(smem + L::kB + stage * (kAresBN / 2) * kBK, &tmap_b, fb, kb * kBK, b_row0);
-                    tma_load_2d_pair_elect(smem + L::kSfb + stage * kSfaBytes, &tmap_sfb, fb, 0,
-                                           2 * (sfb_tile * a.nkb + kb));
-                    ++b_issued;
-                    if (++stage == S) { stage = 0; phase ^= 1u; }
-                }
-            }
-        }
-        if (lane == 0) {        // read by the leader's drain
-            *b_issued_slot = b_issued;
-            *a_units_slot = a_units;
-            *a_kb_slot = a_kb;
-        }
-    } else if (warp == 1) {
-        if (leader) {
-            // ---------------- MMA issuer (leader CTA, for both) ----------------
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            const uint32_t sfa_t = tmem_base + kAresSfCol;
-            const uint32_t sfb_t = sfa_t + 4;
-            int j = 0, ul = 0;
-            for (int u = pair; u < units && ok; u += npairs, ++ul) {
-                for (int i = 0; i < tiles_n && ok; ++i, ++j) {
-                    const int acc = j % 3;
-                    if (j >= 3 && !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(j / 3 - 1) & 1u, abort, a.err,
-                                             a.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d = tmem_base + static_cast<uint32_t>(acc) * kAresAccCols;
-                    for (int kb = 0; kb < a.nkb; ++kb) {
-                        if (i == 0 && !mbar_wait(&a_full[kb], static_cast<uint32_t>(ul) & 1u, abort, a.err,
-                                                 a.timeout_ns)) {
-                            ok = false;
-                            break;
-                        }
-                        if (!mbar_wait(&b_full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
-                        __syncwarp();
-                        tc_fence_after();
-                        tc_cp_pair_elect(sfa_t, sdesc_scale_block(smem_u32(smem + L::kSfa + kb * kSfaBytes)));
-                        tc_cp_pair_elect(sfb_t, sdesc_scale_block(smem_u32(smem + L::kSfb + stage * kSfaBytes)));
-                        const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(smem + L::kA + kb * kBM * kBK));
-                        const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(smem + L::kB + stage * (kAresBN / 2) * kBK));
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            tc_mma_mxf8_pair_elect(d, adesc + 2u * k, bdesc + 2u * k, idesc_mxf8_e4m3(2 * kBM, kAresBN, k),
-                                                   sfa_t | (static_cast<uint32_t>(k) << 30),
-                                                   sfb_t | (static_cast<uint32_t>(k) << 30), (kb | k) != 0 ? 1u : 0u);
-                        }
-                        tc_commit_pair_elect(&b_empty[stage], 0x3);               // both CTAs' stage is free
-                        if (i == tiles_n - 1) tc_commit_pair_elect(&a_empty[kb], 0x3);   // slot kb reusable
-                        if (++stage == S) { stage = 0; phase ^= 1u; }
-                    }
-                    if (!ok) break;
-                    tc_commit_pair_elect(&tmem_full[acc], 0x3);
-                }
-            }
-            __syncwarp();
-            tc_commit_pair_elect(drain, 0x1);
-            mbar_wait_drain(drain, 0, a.timeout_ns);
-        }
-    } else {
-        // ---------------- epilogue (both CTAs) ----------------
-        const int q = warp & 3;             // TMEM lane quadrant this warp may access
-        const int g = (warp - 2) >> 2;      // group: drains every other tile
-        uint8_t* stage = smem + L::kStage + (warp - 2) * kStageBytes;
-        const uint32_t empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-        const uint32_t empty1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-        const uint32_t empty2 = mapa_shared(smem_u32(&acc_empty[2]), 0);
-        int j = 0;
-        bool ok = true;
-        for (int u = pair; u < units && ok; u += npairs) {
-            const AresUnit U = decode_unit(u, rank, a, off, pm128, pm256);
-            for (int i = 0; i < tiles_n; ++i, ++j) {
-                if ((j & 1) != g) continue;
-                const int acc = j % 3;
-                if (!mbar_wait(&tmem_full[acc], static_cast<uint32_t>(j / 3) & 1u, abort, a.err, a.timeout_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                Tile T;
-                T.a_row0 = U.a_row0;
-                T.rows_valid = U.rows_valid;
-                T.n0 = i * kAresBN;
-                T.b_row0 = T.sfa_tile = T.sfb_tile0 = T.sfb_tile1 = 0;
-                epilogue_tile<true, 128, false>(a, T, tmem_base, false, stage, 0u,
-                                                acc == 0 ? empty0 : (acc == 1 ? empty1 : empty2), q, lane,
-                                                static_cast<uint32_t>(acc) * kAresAccCols);
-            }
-        }
-    }
-
-    // Teardown as in the pair kernel: after the first cluster barrier nothing is issued any more; the
-    // leader drains the last fills either CTA issued, of the B ring and of every resident A slot,
-    // supplying the missing half of a fill's transaction count where only one CTA issued it.
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();
-    if (leader && warp == 0 && lane == 0) {
-        const uint32_t mine = *b_issued_slot;
-        const uint32_t peer = ld_shared_cluster_u32(mapa_shared(smem_u32(b_issued_slot), 1));
-        const uint32_t hi = max(mine, peer);
-        for (uint32_t i = hi > static_cast<uint32_t>(S) ? hi - S : 0u; i < hi; ++i) {
-            uint64_t* bar = &b_full[i % S];
-            if (i >= mine)
-                mbar_arrive_expect_tx(bar, kAresBBytes);
-            else if (i >= peer)
-                mbar_complete_tx(bar, kAresBBytes);
-            mbar_wait_drain(bar, (i / S) & 1u, a.timeout_ns);
-        }
-        const uint32_t mu = *a_units_slot, mk = *a_kb_slot;
-        const uint32_t pu = ld_shared_cluster_u32(mapa_shared(smem_u32(a_units_slot), 1));
-        const uint32_t pk = ld_shared_cluster_u32(mapa_shared(smem_u32(a_kb_slot), 1));
-        for (int kb = 0; kb < a.nkb; ++kb) {
-            // Fills of slot kb: every unit begun before the last one, plus the last if it reached kb.
-            const uint32_t fm = mu ? mu - 1 + (static_cast<uint32_t>(kb) < mk ? 1u : 0u) : 0u;
-            const uint32_t fp = pu ? pu - 1 + (static_cast<uint32_t>(kb) < pk ? 1u : 0u) : 0u;
-            const uint32_t fh = max(fm, fp);
-            if (fh == 0) continue;
-            if (fm < fh)
-                mbar_arrive_expect_tx(&a_full[kb], kAresABytes);
-            else if (fp < fh)
-                mbar_complete_tx(&a_full[kb], kAresABytes);
-            mbar_wait_drain(&a_full[kb], (fh - 1) & 1u, a.timeout_ns);
         }
     }
     cluster_sync();

@@ -52,7 +52,6 @@ struct DeviceInfo {
     int qt_blocks_per_sm[4] = {0, 0, 0, 0};   // TMA-staged quantizer, by direction bits
     int ge_blocks_per_sm = 1;
     int pair_clusters[2] = {0, 0};    // co-resident 2-CTA clusters of the pair GEMM (dense, grouped)
-    int ares_clusters = 0;            // ... of the short-K grouped kernel
     bool ok = false;
 };
 
@@ -78,8 +77,7 @@ int max_pair_clusters(K kernel, int smem, int sms) {
     return n;
 }
 
-// GEMM kernel selection: 0 = CTA-pair kernels (default; grouped GEMMs with K <= 768 take the
-// resident-A kernel), 1 = single-CTA kernel, 2 = the general CTA-pair kernel for every shape.
+// GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
 std::atomic<int> g_gemm_variant{0};
 // Quantizer selection: 0 = register-staged tiles (default; columnwise-only calls take the TMA-staged
 // kernel, measured faster for that direction), 1 = TMA-staged tiles.
@@ -154,13 +152,10 @@ const DeviceInfo* device_info() {
             cudaFuncSetAttribute(mx_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmPairSmemGrouped) != cudaSuccess ||
             cudaFuncSetAttribute(mx_gemm_pair_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmPairSmemGrouped) != cudaSuccess ||
-            cudaFuncSetAttribute(mx_gemm_ares_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmAresSmem) != cudaSuccess)
+                                 kGemmPairSmemGrouped) != cudaSuccess)
             return nullptr;
         d.pair_clusters[0] = max_pair_clusters(mx_gemm_pair_kernel<false>, kGemmPairSmemDense, d.sms);
         d.pair_clusters[1] = max_pair_clusters(mx_gemm_pair_kernel<true>, kGemmPairSmemGrouped, d.sms);
-        d.ares_clusters = max_pair_clusters(mx_gemm_ares_kernel, kGemmAresSmem, d.sms);
         d.ok = true;
     }
     return &d;
@@ -275,30 +270,6 @@ int vector_store_ok(const void* c, int64_t ld_c, mx_out_dtype dt) {
 // copies count on the leader's barrier).
 bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t blocks) {
     return encode_2d(map, 1, base, 256, static_cast<uint64_t>(2 * blocks), 256, 256, 2);
-}
-
-using PairKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
-
-// Launches a CTA-pair GEMM kernel with a cluster dimension of 2.
-mx_status launch_pair_kernel(PairKernel kernel, int smem, int pairs, const CUtensorMap& ta, const CUtensorMap& tb,
-                             const CUtensorMap& tsa, const CUtensorMap& tsb, const GemmArgs& a, mx_stream stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsa, tsb, a) != cudaSuccess) {
-        cudaGetLastError();
-        return MX_ERR_CUDA;
-    }
-    return launched();
 }
 
 // Launches the CTA-pair GEMM with a cluster dimension of 2.
@@ -656,7 +627,7 @@ mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, c
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    const bool pair = g_gemm_variant.load() != 1;
+    const bool pair = g_gemm_variant.load() == 0;
     GemmArgs a{};
     a.sfa = sa_swz;
     a.sfb = sb_swz;
@@ -707,8 +678,7 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     if (empty) return MX_OK;
     const DeviceInfo* d = nullptr;
     if (mx_status st = check_device(&d)) return st;
-    const int variant = g_gemm_variant.load();
-    const bool pair = variant != 1;
+    const bool pair = g_gemm_variant.load() == 0;
     GemmArgs a{};
     a.sfa = sa_swz;
     a.sfb = sb_swz;
@@ -729,19 +699,6 @@ mx_status mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_
     a.err = d->status;
     a.timeout_ns = g_timeout_ns.load();
     CUtensorMap ta, tb;
-    if (variant == 0 && a.nkb <= kAresMaxKb) {
-        // Short K: resident A, 128-column tiles. Upper bound on units: every group adds at most one
-        // partial 256-row m-tile.
-        a.tiles_n = static_cast<int>(ceil_div(N, kAresBN));
-        CUtensorMap tsa, tsb;
-        if (!make_tmap(&ta, qa, K, total_rows, kBK, kBM) || !make_tmap(&tb, qb, K, G * N, kBK, kAresBN / 2) ||
-            !make_tmap_sf(&tsa, sa_swz, (ceil_div(total_rows, 128) + G) * a.nkb) ||
-            !make_tmap_sf(&tsb, sb_swz, G * a.n_rowtiles * a.nkb))
-            return MX_ERR_CUDA;
-        const int64_t max_units = ceil_div(total_rows, 2 * kBM) + G;
-        const int pairs = static_cast<int>(std::min<int64_t>(max_units, d->ares_clusters));
-        return launch_pair_kernel(mx_gemm_ares_kernel, kGemmAresSmem, pairs, ta, tb, tsa, tsb, a, stream);
-    }
     if (pair) {
         // Upper bounds: every group adds at most one partial 256-row tile, one partial 128-row scale tile.
         const int64_t max_tiles = (ceil_div(total_rows, 2 * kBM) + G) * a.tiles_n;
@@ -837,7 +794,7 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
     return launched();
 }
 
-void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 || variant == 2 ? variant : 0); }
+void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
 
 void mx_set_quantize_variant(int variant) { g_quant_variant.store(variant == 1 ? 1 : 0); }
 

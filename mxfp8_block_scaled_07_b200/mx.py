@@ -295,12 +295,11 @@ def set_wait_timeout_ns(ns: int):
     lib().mx_set_wait_timeout_ns(int(ns))
 
 
-GEMM_PAIR, GEMM_SINGLE, GEMM_PAIR_ONLY = 0, 1, 2
+GEMM_PAIR, GEMM_SINGLE = 0, 1
 
 
 def set_gemm_variant(variant: int):
-    """0: CTA-pair kernels (default; grouped GEMMs with K <= 768 keep A resident); 1: single-CTA
-    kernel; 2: the 256 x 256 CTA-pair kernel for every shape."""
+    """0: CTA-pair GEMM kernel (default); 1: single-CTA kernel."""
     lib().mx_set_gemm_variant(int(variant))
 
 

@@ -45,6 +45,10 @@ def grouped_case(counts, N, K, out_dtype, seed=0, device_inputs=None):
     qx, sx_raw, _, _ = mx.quantize(Xd, True, False, swizzle=False)
     sx = mx.swizzle_scales(sx_raw, counts)
     qw, sw, _, _ = mx.quantize(Wd.reshape(G * N, K), True, False, swizzle=True)
+    if N % 128:
+        # B's scales are G consecutive per-expert layouts, each padded to 128 rows on its own; one
+        # layout of all G * N rows matches that only when N is a multiple of 128.
+        sw = torch.cat([mx.quantize(Wd[g].contiguous(), True, False, swizzle=True)[1] for g in range(G)])
     offs = torch.tensor(off, dtype=torch.int32, device="cuda")
     c = mx.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw, offs, out_dtype=out_dtype)
     torch.cuda.synchronize()
@@ -104,8 +108,8 @@ def test_moe_layer_full_size_sampled():
 @pytest.mark.parametrize("K", [32, 128, 384, 768, 896])
 @pytest.mark.parametrize("N", [128, 200, 640])
 def test_grouped_short_k_shapes(K, N, grouped_variant):
-    """Around the resident-A kernel's range (K <= 768: 1..6 resident k-blocks; 896 falls back to the
-    pair kernel) with N not a multiple of 128 and experts of 0, 1, 128, 255, 256 and 300 rows."""
+    """Short K (1 to 7 k-blocks of 128, the MoE down projection's 768 among them) with N not a
+    multiple of 128 and experts of 0, 1, 128, 255, 256 and 300 rows."""
     counts = [128, 0, 1, 300, 255, 256, 3]
     X, W, off, c = grouped_case(counts, N, K, torch.float32, seed=K + N)
     qx, sx = oracle.quantize_rowwise(X)
@@ -116,8 +120,7 @@ def test_grouped_short_k_shapes(K, N, grouped_variant):
 
 
 def test_grouped_many_units_per_pair():
-    """More m-tiles than CTA pairs (each pair walks several units, so resident A slots are refilled
-    while B of the previous unit is still in flight), 40 experts of up to 700 rows, K = 768."""
+    """More 256-row tiles per expert than one, across many experts of up to 700 rows, K = 768."""
     g = np.random.default_rng(11)
     counts = [int(c) for c in g.integers(0, 700, 40)]
     N, K = 384, 768
