@@ -917,7 +917,7 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
     return out
 
 
-CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
+CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-dy-col", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
          "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up")
 SUBSET_LAYERS = 2      # quant-sync-subset: the first 2 layers' 8 weights (0.39 G elements, ~1.2 GB on the device)
 
@@ -950,6 +950,10 @@ def run_case(name: str, reps: int):
         _, _, x = synth.update_inputs(device=dev)
         bufs = mx.quantize(x, True, True)
         fn = lambda: mx.quantize(x, True, True, out=bufs)
+    elif name == "quant-dy-col":
+        _, _, x = synth.update_inputs(device=dev)
+        bufs = mx.quantize(x, False, True)
+        fn = lambda: mx.quantize(x, False, True, out=bufs)
     elif name == "grid-equal-gate-up":
         x = synth.sync_weight(0, 2, device=dev)
         q, _, _, _ = mx.quantize(x, True, False)
