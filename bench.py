@@ -565,13 +565,37 @@ def scaled_mm_fn(qa, sa, qb, sb):
         return None
 
 
-def cublas_line(fn, flops, reps, flush, stream) -> dict:
+def scaled_grouped_mm_fn(qa, sa_grp, qb, sb, row_offsets):
+    """torch `scaled_grouped_mm` (MXFP8, BlockWise1x32 scales in the SWIZZLE_32_4_4 layout) on this
+    library's bytes: A [rows, K] with its grouped scale layout (each expert padded to 128 rows) as a
+    2-D [padded rows, padded K/32] tensor, B [G, N, K] seen as [G, K, N] with its G per-expert
+    layouts as [G, bytes per expert]; group ends from the row offsets. None if torch lacks it."""
+    import torch
+    import torch.nn.functional as F
+
+    try:
+        G, N, K = qb.shape
+        kb_pad = (K // 32 + 3) // 4 * 4
+        fa, fb = qa.view(torch.float8_e4m3fn), qb.view(torch.float8_e4m3fn).transpose(-2, -1)
+        ea = sa_grp.view(torch.float8_e8m0fnu).reshape(-1, kb_pad)
+        eb = sb.view(torch.float8_e8m0fnu).reshape(G, -1)
+        ends = row_offsets[1:].contiguous()
+        return lambda: F.scaled_grouped_mm(fa, fb, ea, F.ScalingType.BlockWise1x32, eb, F.ScalingType.BlockWise1x32,
+                                           swizzle_a=F.SwizzleType.SWIZZLE_32_4_4,
+                                           swizzle_b=F.SwizzleType.SWIZZLE_32_4_4, offs=ends,
+                                           output_dtype=torch.bfloat16)
+    except (AttributeError, TypeError):
+        return None
+
+
+def cublas_line(fn, flops, reps, flush, stream, key="cublas") -> dict:
+    """Times a library MXFP8 GEMM on the same bytes; keys <key>_mxfp8_tflops / <key>_ms."""
     try:
         fn()
         ms = time_gpu(fn, reps, flush, stream)
-        return {"cublas_mxfp8_tflops": round(flops / (ms * 1e-3) / 1e12, 1), "cublas_ms": round(ms, 4)}
+        return {f"{key}_mxfp8_tflops": round(flops / (ms * 1e-3) / 1e12, 1), f"{key}_ms": round(ms, 4)}
     except (RuntimeError, TypeError, NotImplementedError) as e:
-        return {"cublas_mxfp8_tflops": None, "cublas_note": f"torch scaled_mm MXFP8 unavailable: {type(e).__name__}"}
+        return {f"{key}_mxfp8_tflops": None, f"{key}_note": f"torch MXFP8 GEMM unavailable: {type(e).__name__}"}
 
 
 def guarded(fn):
@@ -596,7 +620,7 @@ def run_secondary(device, peaks, reps=10):
            "fp8_peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
            "spec_fp8_tflops": 4500.0}
 
-    def add_gemm(name, flops, fn, lib_fn=None):
+    def add_gemm(name, flops, fn, lib_fn=None, lib_key="cublas"):
         for _ in range(2):
             fn()
         mx.device_error()                     # clear before the timed launches
@@ -606,10 +630,10 @@ def run_secondary(device, peaks, reps=10):
                "frac_of_fp8_peak": round(tf / fp8_peak, 3), "frac_of_spec_4500": round(tf / 4500.0, 3)}
         rec.update(device_status())
         if lib_fn is not None:
-            lib = cublas_line(lib_fn, flops, reps, flush, stream)
+            lib = cublas_line(lib_fn, flops, reps, flush, stream, lib_key)
             rec.update(lib)
-            if lib.get("cublas_mxfp8_tflops"):
-                rec["mx_over_cublas"] = round(tf / lib["cublas_mxfp8_tflops"], 3)
+            if lib.get(f"{lib_key}_mxfp8_tflops"):
+                rec[f"mx_over_{lib_key}"] = round(tf / lib[f"{lib_key}_mxfp8_tflops"], 3)
         out["gemm"].append(rec)
 
     def add_quant(name, x, row, col):
@@ -669,7 +693,8 @@ def run_secondary(device, peaks, reps=10):
         qb = qb.reshape(G, N, K)
         C = torch.empty((rows, N), dtype=torch.bfloat16, device=device)
         add_gemm(f"{name} grouped {rows}x{N}x{K} (128 experts)", 2.0 * rows * N * K,
-                 lambda: mx.grouped_gemm(qa, sa, qb, sb, offs, out=C))
+                 lambda: mx.grouped_gemm(qa, sa, qb, sb, offs, out=C), scaled_grouped_mm_fn(qa, sa, qb, sb, offs),
+                 "torch_grouped")
         del qa, sa_raw, sa, qb, sb, C
     # FP8-blockwise grids of one weight (128 x 128 blocks): FP32 scales (the sampler's) against
     # power-of-two scales (the learner's on SM100), beside the MXFP8 grid both sides share here.

@@ -130,3 +130,36 @@ def test_grouped_many_units_per_pair():
     G = len(counts)
     ref, abs_sum = oracle.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw.reshape(G, N, K // 32), off)
     assert_gemm_close(to_np(c.float()), ref, abs_sum, True, "grouped many units")
+
+
+def test_library_cross_check_scaled_grouped_mm_blockwise_1x32():
+    """torch's grouped MXFP8 GEMM (scaled_grouped_mm, BlockWise1x32 + SWIZZLE_32_4_4) fed with this
+    library's bytes, A's grouped scale layout (each expert padded to 128 rows) and B's per-expert
+    layouts must agree with the oracle as well: an independent consumer of the grouped layout."""
+    import torch.nn.functional as F
+
+    counts = [0, 5, 128, 129, 300, 0, 1, 64, 256, 257]
+    N, K = 256, 384
+    X, W, off, c = grouped_case(counts, N, K, torch.bfloat16, seed=21)
+    G = len(counts)
+    Xd, Wd = X.cuda(), W.cuda()
+    qx, sx_raw, _, _ = mx.quantize(Xd, True, False, swizzle=False)
+    sx = mx.swizzle_scales(sx_raw, counts)
+    qw, sw, _, _ = mx.quantize(Wd.reshape(G * N, K), True, False, swizzle=True)
+    kb_pad = (K // 32 + 3) // 4 * 4
+    ends = torch.tensor(off[1:], dtype=torch.int32, device="cuda")
+    try:
+        lib = F.scaled_grouped_mm(qx.view(torch.float8_e4m3fn),
+                                  qw.view(torch.float8_e4m3fn).reshape(G, N, K).transpose(-2, -1),
+                                  sx.view(torch.float8_e8m0fnu).reshape(-1, kb_pad), F.ScalingType.BlockWise1x32,
+                                  sw.view(torch.float8_e8m0fnu).reshape(G, -1), F.ScalingType.BlockWise1x32,
+                                  swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                                  offs=ends, output_dtype=torch.bfloat16)
+    except (RuntimeError, TypeError, NotImplementedError, AttributeError) as e:  # pragma: no cover
+        pytest.skip(f"torch scaled_grouped_mm MXFP8 path unavailable: {e}")
+    torch.cuda.synchronize()
+    qxo, sxo = oracle.quantize_rowwise(X)
+    qwo, swo = oracle.quantize_rowwise(W.reshape(-1, K))
+    ref, abs_sum = oracle.grouped_gemm(qxo, sxo, qwo.reshape(G, N, K), swo.reshape(G, N, K // 32), off)
+    assert_gemm_close(to_np(lib.float()), ref, abs_sum, True, "torch scaled_grouped_mm on our layouts")
+    assert_gemm_close(to_np(c.float()), ref, abs_sum, True, "mx_grouped_gemm")
