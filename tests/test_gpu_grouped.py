@@ -105,8 +105,7 @@ def test_moe_layer_full_size_sampled():
                               ref, abs_sum, True, f"{name} expert {e}")
 
 
-@pytest.mark.parametrize("K", [32, 128, 384, 768, 896])
-@pytest.mark.parametrize("N", [128, 200, 640])
+@pytest.mark.parametrize("K,N", [(32, 200), (128, 640), (384, 200), (768, 200), (768, 640), (896, 128)])
 def test_grouped_short_k_shapes(K, N, grouped_variant):
     """Short K (1 to 7 k-blocks of 128, the MoE down projection's 768 among them) with N not a
     multiple of 128 and experts of 0, 1, 128, 255, 256 and 300 rows."""
@@ -122,7 +121,7 @@ def test_grouped_short_k_shapes(K, N, grouped_variant):
 def test_grouped_many_units_per_pair():
     """More 256-row tiles per expert than one, across many experts of up to 700 rows, K = 768."""
     g = np.random.default_rng(11)
-    counts = [int(c) for c in g.integers(0, 700, 40)]
+    counts = [int(c) for c in g.integers(0, 600, 24)]
     N, K = 384, 768
     X, W, off, c = grouped_case(counts, N, K, torch.bfloat16, seed=5)
     qx, sx = oracle.quantize_rowwise(X)
