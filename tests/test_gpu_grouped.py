@@ -131,6 +131,46 @@ def test_grouped_many_units_per_pair():
     assert_gemm_close(to_np(c.float()), ref, abs_sum, True, "grouped many units")
 
 
+def test_expired_waits_end_the_grouped_gemm_cleanly(grouped_variant):
+    """With a 1 ns deadline every wait that does not succeed at once expires: the grouped kernel
+    records error bit 1, drains its copies and MMAs and returns; the next grouped GEMM is exact. A
+    wait's first try may itself block for a while (the hardware's suspend window), so K is long
+    enough for the tiles to outlast it, and the launch is repeated until a wait has expired."""
+    expired_waits_case(8192)
+
+
+def expired_waits_case(K):
+    g = np.random.default_rng(12)
+    counts = [int(c) for c in g.integers(0, 2000, 40)]
+    G, N = len(counts), 1024
+    X = synth.normal_bf16((sum(counts), K), seed=6).cuda()
+    W = synth.normal_bf16((G, N, K), std=0.02, seed=7).cuda()
+    qx, sx_raw, _, _ = mx.quantize(X, True, False, swizzle=False)
+    sx = mx.swizzle_scales(sx_raw, counts)
+    qw, sw, _, _ = mx.quantize(W.reshape(G * N, K), True, False, swizzle=True)
+    offs = torch.tensor(synth.group_offsets(counts), dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    assert mx.device_error() == 0
+    mx.set_wait_timeout_ns(1)
+    try:
+        for _ in range(8):
+            mx.grouped_gemm(qx, sx, qw.reshape(G, N, K), sw, offs, out_dtype=torch.bfloat16)
+            torch.cuda.synchronize()
+            bits = mx.device_error()
+            if bits:
+                break
+    finally:
+        mx.set_wait_timeout_ns(0)
+    assert bits == 1
+    counts = [3, 0, 300, 129]
+    X, W, off, c = grouped_case(counts, 256, 384, torch.float32, seed=7)
+    qx, sx = oracle.quantize_rowwise(X)
+    qw, sw = oracle.quantize_rowwise(W.reshape(-1, 384))
+    ref, abs_sum = oracle.grouped_gemm(qx, sx, qw.reshape(4, 256, 384), sw.reshape(4, 256, 384 // 32), off)
+    assert_gemm_close(to_np(c), ref, abs_sum, False, "grouped after expired waits")
+    assert mx.device_error() == 0
+
+
 def test_library_cross_check_scaled_grouped_mm_blockwise_1x32():
     """torch's grouped MXFP8 GEMM (scaled_grouped_mm, BlockWise1x32 + SWIZZLE_32_4_4) fed with this
     library's bytes, A's grouped scale layout (each expert padded to 128 rows) and B's per-expert
