@@ -616,7 +616,7 @@ def run_secondary(device, peaks, reps=10):
     stream = torch.cuda.current_stream()
     flush = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=device)   # 2 x (2 x L2)
     fp8_peak = peaks["bf16_tflops"] * NOMINAL_FP8_OVER_BF16
-    out = {"gemm": [], "quantize": [], "fp8_peak_tflops": round(fp8_peak, 1),
+    out = {"gemm": [], "quantize": [], "swizzle": [], "fp8_peak_tflops": round(fp8_peak, 1),
            "fp8_peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
            "spec_fp8_tflops": 4500.0}
 
@@ -650,9 +650,22 @@ def run_secondary(device, peaks, reps=10):
         rec.update(device_status())
         out["quantize"].append(rec)
 
+    def add_swizzle(name, s_raw, groups=None):
+        """Standalone scale rearrangement (Table 6): raw scales read once, the layout written once."""
+        o = mx.swizzle_scales(s_raw, groups)
+        fn = lambda: mx.swizzle_scales(s_raw, groups, out=o)
+        fn()
+        mx.device_error()
+        ms = time_gpu(fn, reps, flush, stream)
+        gbs = (s_raw.numel() + o.numel()) / (ms * 1e-3) / 1e9
+        rec = {"workload": name, "gbs": round(gbs, 1), "ms": round(ms, 4), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        rec.update(device_status())
+        out["swizzle"].append(rec)
+
     # Dense forward linear (Table 5 micro-batch token counts) against gate_up.
     W = synth.sync_weight(0, 2, device=device)
     qw, sw, _, _ = mx.quantize(W, True, False)
+    add_swizzle("gate_up weight scales 24576x128", mx.quantize(W, True, False, swizzle=False)[1])
     for M in synth.FWD_TOKENS:
         X = synth.fwd_activations(M, device=device)
         add_quant(f"fwd activations {M}x4096 rowwise", X, True, False)
@@ -689,6 +702,8 @@ def run_secondary(device, peaks, reps=10):
         G, N, K = Wt.shape
         qa, sa_raw, _, _ = mx.quantize(A, True, False, swizzle=False)
         sa = mx.swizzle_scales(sa_raw, counts)
+        add_swizzle(f"{name} A scales {rows}x{K // 32} grouped (128 experts, each padded to 128 rows)", sa_raw,
+                    counts)
         qb, sb, _, _ = mx.quantize(Wt.reshape(G * N, K), True, False)
         qb = qb.reshape(G, N, K)
         C = torch.empty((rows, N), dtype=torch.bfloat16, device=device)
@@ -943,7 +958,8 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
 
 
 CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-dy-col", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
-         "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up")
+         "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up",
+         "swizzle-moe-gate-up", "swizzle-moe-down")
 SUBSET_LAYERS = 2      # quant-sync-subset: the first 2 layers' 8 weights (0.39 G elements, ~1.2 GB on the device)
 
 
@@ -984,6 +1000,14 @@ def run_case(name: str, reps: int):
         q, _, _, _ = mx.quantize(x, True, False)
         q2 = q.clone()
         fn = lambda: mx.grid_equal(q, q2)
+    elif name.startswith("swizzle-moe"):
+        # The grouped A-operand scale layout of the MoE GEMMs (raw scales of X_perm or H).
+        counts, Xp, Hh, _, _ = synth.moe_inputs(device=dev)
+        counts = [int(c) for c in counts]
+        _, s_raw, _, _ = mx.quantize(Xp if name == "swizzle-moe-gate-up" else Hh, True, False, swizzle=False)
+        del Xp, Hh
+        o = mx.swizzle_scales(s_raw, counts)
+        fn = lambda: mx.swizzle_scales(s_raw, counts, out=o)
     elif name.startswith("gemm-moe"):
         counts, Xp, Hh, W1, W2 = synth.moe_inputs(device=dev)
         counts = [int(c) for c in counts]

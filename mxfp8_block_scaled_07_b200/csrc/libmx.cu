@@ -557,12 +557,14 @@ mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, con
     const int64_t* gr = group_rows_host ? group_rows_host : &one;
     const int64_t ng = group_rows_host ? groups : 1;
     const int64_t ctiles = ceil_div(kblocks, 4);
+    const bool quad = kblocks % 16 == 0 && aligned16(s);
     int64_t src_row = 0, out_block = 0;
     for (int64_t g0 = 0; g0 < ng; g0 += kSwzMaxGroups) {
         SwizzleArgs a;
         a.s = s;
         a.kblocks = kblocks;
         a.ctiles = ctiles;
+        a.word_loads = kblocks % 4 == 0 && (reinterpret_cast<uintptr_t>(s) & 3u) == 0;
         a.ngroups = static_cast<int>(std::min<int64_t>(kSwzMaxGroups, ng - g0));
         a.out = s_swz + out_block * 512;
         int64_t local_block = 0;
@@ -575,9 +577,12 @@ mx_status mx_swizzle_scales(const uint8_t* s, int64_t rows, int64_t kblocks, con
         }
         a.block_start[a.ngroups] = local_block;
         if (local_block > 0) {
-            const int64_t warps = local_block;
+            const int64_t warps = quad ? local_block / 4 : local_block;
             const int64_t grid = std::min<int64_t>(ceil_div(warps * 32, 256), int64_t(d->sms) * 16);
-            swizzle_kernel<<<grid, 256, 0, stream>>>(a);
+            if (quad)
+                swizzle_kernel<true><<<grid, 256, 0, stream>>>(a);
+            else
+                swizzle_kernel<false><<<grid, 256, 0, stream>>>(a);
             if (mx_status st = launched()) return st;
         }
         out_block += local_block;

@@ -11,7 +11,9 @@ from mxfp8_block_scaled_07_b200 import mx, synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("rows,kb", [(1, 1), (128, 4), (300, 13), (1024, 64), (4097, 130)])
+# kb % 16 == 0 takes the 16-byte-load kernel, kb % 4 == 0 the 32-bit-load one, the rest byte loads.
+@pytest.mark.parametrize("rows,kb", [(1, 1), (128, 4), (300, 13), (1024, 64), (4097, 130), (1000, 24), (513, 32),
+                                     (777, 48)])
 def test_swizzle_single_group(rows, kb):
     s = synth.random_bytes(rows * kb, seed=rows + kb).reshape(rows, kb)
     out = mx.swizzle_scales(s.cuda())
@@ -19,9 +21,22 @@ def test_swizzle_single_group(rows, kb):
     assert np.array_equal(to_np(out), oracle.swizzle(s.numpy()))
 
 
-@pytest.mark.parametrize("groups", [[0, 5, 128, 129, 300, 0, 1], [7] * 200, [0], [256, 0, 0, 3]])
-def test_swizzle_grouped(groups):
-    kb = 64
+@pytest.mark.parametrize("offset", [1, 4])
+def test_swizzle_unaligned_source(offset):
+    """A raw-scale pointer that is not 16-byte (or not 4-byte) aligned takes the narrower loads."""
+    rows, kb = 300, 64
+    s = synth.random_bytes(rows * kb, seed=9).reshape(rows, kb)
+    buf = torch.zeros(rows * kb + 16, dtype=torch.uint8, device="cuda")
+    buf[offset:offset + rows * kb] = s.reshape(-1).cuda()
+    out = mx.swizzle_scales(buf[offset:offset + rows * kb].view(rows, kb))
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(out), oracle.swizzle(s.numpy()))
+
+
+@pytest.mark.parametrize("groups,kb", [([0, 5, 128, 129, 300, 0, 1], 64), ([7] * 200, 64), ([0], 64),
+                                       ([256, 0, 0, 3], 64), ([0, 5, 128, 129, 300, 0, 1], 24),
+                                       ([130, 0, 1, 255], 13)])
+def test_swizzle_grouped(groups, kb):
     rows = sum(groups)
     s = synth.random_bytes(max(rows, 1) * kb, seed=len(groups))[: rows * kb].reshape(rows, kb)
     if rows == 0:
