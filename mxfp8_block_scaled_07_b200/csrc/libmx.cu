@@ -794,8 +794,10 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
     a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (ld_x % 16 == 0) &&
               (reinterpret_cast<uintptr_t>(q) % 32 == 0);
     const int64_t tiles = int64_t(a.tiles_m) * a.tiles_k;
-    const int64_t grid = std::min<int64_t>(tiles, int64_t(d->sms) * 4);
-    quantize_block128_kernel<<<grid, kQThreads, 0, stream>>>(a);
+    if (a.pow2)
+        quantize_block128_kernel<true><<<std::min<int64_t>(tiles, int64_t(d->sms) * 2), kQThreads, 0, stream>>>(a);
+    else
+        quantize_block128_kernel<false><<<std::min<int64_t>(tiles, int64_t(d->sms) * 4), kQThreads, 0, stream>>>(a);
     return launched();
 }
 
