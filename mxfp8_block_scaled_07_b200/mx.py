@@ -104,7 +104,10 @@ def swizzled_scale_bytes(rows: int, kblocks: int) -> int:
 
 
 def grouped_swizzled_scale_bytes(group_rows, kblocks: int) -> int:
-    return sum(swizzled_scale_bytes(int(r), kblocks) for r in group_rows)
+    """Bytes of the grouped layout: every group padded to 128 rows on its own (no library call per
+    group: the padded row count times the padded K-block count)."""
+    rows = sum((int(r) + 127) // 128 * 128 for r in group_rows)
+    return swizzled_scale_bytes(rows, kblocks) if rows else 0
 
 
 def quantize(x: torch.Tensor, rowwise: bool = True, colwise: bool = False, swizzle: bool = True, out=None):
@@ -192,12 +195,12 @@ def swizzle_scales(s: torch.Tensor, group_rows=None, out=None):
     rows, kb = s.shape
     if group_rows is not None:
         gr = [int(r) for r in group_rows]
-        size = grouped_swizzled_scale_bytes(gr, kb)
         arr = (ctypes.c_int64 * len(gr))(*gr)
         gptr, ng = ctypes.cast(arr, ctypes.c_void_p), len(gr)
     else:
-        size, gptr, ng = swizzled_scale_bytes(rows, kb), None, 0
+        gr, gptr, ng = None, None, 0
     if out is None:
+        size = grouped_swizzled_scale_bytes(gr, kb) if gr is not None else swizzled_scale_bytes(rows, kb)
         out = torch.empty(size, dtype=torch.uint8, device=s.device)
     st = lib().mx_swizzle_scales(_p(s), rows, kb, gptr, ng, _p(out), ctypes.c_void_p(_stream(s.device)))
     _check(st, "mx_swizzle_scales")

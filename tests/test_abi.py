@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from mxfp8_block_scaled_07_b200 import build as mxbuild
@@ -55,6 +56,18 @@ def test_swizzled_scale_bytes(L):
 
 FAKE = ctypes.c_void_p(0x10000)       # never dereferenced: every call below fails validation first
 FAKE_ODD = ctypes.c_void_p(0x10008)
+
+
+def test_grouped_scale_bytes_match_per_group_layouts(L):
+    """The binding's grouped size (padded rows summed once) equals the sum of the library's size
+    of every group's own layout."""
+    from mxfp8_block_scaled_07_b200 import mx
+
+    g = np.random.default_rng(3)
+    for _ in range(100):
+        groups = [int(r) for r in g.choice([0, 1, 127, 128, 129, 255, 256, 300, 1000], g.integers(1, 20))]
+        kb = int(g.choice([1, 3, 4, 13, 24, 64, 130]))
+        assert mx.grouped_swizzled_scale_bytes(groups, kb) == sum(L.mx_swizzled_scale_bytes(r, kb) for r in groups)
 
 
 def test_quantize_argument_errors(L):
