@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -194,9 +195,8 @@ def swizzle_scales(s: torch.Tensor, group_rows=None, out=None):
     assert s.dtype == torch.uint8 and s.dim() == 2 and s.is_contiguous()
     rows, kb = s.shape
     if group_rows is not None:
-        gr = [int(r) for r in group_rows]
-        arr = (ctypes.c_int64 * len(gr))(*gr)
-        gptr, ng = ctypes.cast(arr, ctypes.c_void_p), len(gr)
+        gr = np.ascontiguousarray(np.asarray(group_rows, dtype=np.int64))       # host memory, read during the call
+        gptr, ng = ctypes.c_void_p(gr.ctypes.data), int(gr.size)
     else:
         gr, gptr, ng = None, None, 0
     if out is None:
