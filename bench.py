@@ -959,7 +959,7 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
 
 CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-dy-col", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
          "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up",
-         "swizzle-moe-gate-up", "swizzle-moe-down")
+         "swizzle-moe-gate-up", "swizzle-moe-down", "block128-pow2-gate-up", "block128-fp32-gate-up")
 SUBSET_LAYERS = 2      # quant-sync-subset: the first 2 layers' 8 weights (0.39 G elements, ~1.2 GB on the device)
 
 
@@ -1000,6 +1000,11 @@ def run_case(name: str, reps: int):
         q, _, _, _ = mx.quantize(x, True, False)
         q2 = q.clone()
         fn = lambda: mx.grid_equal(q, q2)
+    elif name.startswith("block128"):
+        x = synth.sync_weight(0, 2, device=dev)
+        pow2 = name == "block128-pow2-gate-up"
+        g = mx.quantize_block128(x, pow2)
+        fn = lambda: mx.quantize_block128(x, pow2, out=g)
     elif name.startswith("swizzle-moe"):
         # The grouped A-operand scale layout of the MoE GEMMs (raw scales of X_perm or H).
         counts, Xp, Hh, _, _ = synth.moe_inputs(device=dev)
