@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
     const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
     const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
     const int64_t t_end = min(a.total_tiles, t_begin + per);
-    Block32 cur[2], nxt[2];
+    Block32 cur[2];
     TileRef rc, rn;
     if (t_begin < t_end) {
         rc = decode_qtile(a, t_begin);
@@ -405,7 +405,6 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
             rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
             rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
             rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
-            load_row_tile(a, rn, nxt, tid);
         }
         const QTensor& T = a.t[rc.i];
         const int kb = tid & 3;
@@ -449,6 +448,9 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
                 atom_row[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
             }
         }
+        // The tile is in shared memory now: the next tile's loads go into the same registers and
+        // stay in flight through the column pass.
+        if (t + 1 < t_end) load_row_tile(a, rn, cur, tid);
         __syncthreads();
         {
             const int cp = tid & 63;                     // column pair: tile columns 2 cp, 2 cp + 1
@@ -514,8 +516,6 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
             }
         }
         __syncthreads();
-        cur[0] = nxt[0];
-        cur[1] = nxt[1];
         rc = rn;
     }
 }
