@@ -218,9 +218,12 @@ void mx_set_gemm_variant(int variant);
  * 0 (default) loads each thread's two 32-element blocks of a 128 x 128 BF16 tile into registers
  * with 256-bit loads, one tile ahead of the compute (the columnwise pass of a row + col call goes
  * through a swizzled shared-memory copy of the tile), except that columnwise-only calls take the
- * TMA-staged kernel; 1 stages the tiles of every call in shared memory with TMA tensor loads
- * running three tiles ahead. Both produce the same bytes; the default picks the kernel measured
- * faster on B200 for each direction. Other values select 0.
+ * TMA-staged kernel, and rowwise-only calls whose CTAs each walk many tiles (at least 64) take a
+ * split-load form that loads each half of the next tile as soon as the same half of the current
+ * one is encoded; 1 stages the tiles of every call in shared memory with TMA tensor loads running
+ * three tiles ahead; 2 is 0 with the split-load form for every rowwise-only call. All produce the
+ * same bytes; the default picks the kernel measured faster on B200 for each direction and size.
+ * Other values select 0.
  */
 void mx_set_quantize_variant(int variant);
 

@@ -80,7 +80,10 @@ int max_pair_clusters(K kernel, int smem, int sms) {
 // GEMM kernel selection: 0 = CTA-pair kernel (default), 1 = single-CTA kernel.
 std::atomic<int> g_gemm_variant{0};
 // Quantizer selection: 0 = register-staged tiles (default; columnwise-only calls take the TMA-staged
-// kernel, measured faster for that direction), 1 = TMA-staged tiles.
+// kernel, measured faster for that direction; rowwise-only calls whose CTAs each walk at least
+// kSplitTilesPerCta tiles take the split-load form), 1 = TMA-staged tiles, 2 = as 0 with the
+// split-load form for every rowwise-only call.
+constexpr int64_t kSplitTilesPerCta = 64;
 std::atomic<int> g_quant_variant{0};
 
 bool use_tma_quantizer(bool row, bool col) { return g_quant_variant.load() == 1 || (col && !row); }
@@ -133,8 +136,12 @@ const DeviceInfo* device_info() {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
         d.status = static_cast<uint32_t*>(p);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1], quantize_rowwise_kernel<kQMaxTensors>,
+        int split_blocks = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1],
+                                                      quantize_rowwise_kernel<kQMaxTensors, false>, kQThreads, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&split_blocks, quantize_rowwise_kernel<kQMaxTensors, true>,
                                                       kQThreads, 0);
+        d.quant_blocks_per_sm[1] = std::min(d.quant_blocks_per_sm[1], split_blocks);
         if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
         d.quant_blocks_per_sm[3] = quant_occupancy<true>();
         if (!qt_setup<true, false>(&d.qt_blocks_per_sm[1]) || !qt_setup<false, true>(&d.qt_blocks_per_sm[2]) ||
@@ -387,10 +394,13 @@ mx_status launch_quant(const QuantArgs<NT>& a, bool row, bool col, const DeviceI
     if (a.total_tiles == 0) return MX_OK;
     const int which = (row ? 1 : 0) | (col ? 2 : 0);
     const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->quant_blocks_per_sm[which]);
+    const int v = g_quant_variant.load();
     if (col)     // row + col (columnwise only takes the TMA-staged kernel)
         quantize_rowcol_kernel<true, NT><<<grid, kQThreads, 0, stream>>>(a);
+    else if (v == 2 || (v == 0 && a.total_tiles >= kSplitTilesPerCta * grid))
+        quantize_rowwise_kernel<NT, true><<<grid, kQThreads, 0, stream>>>(a);
     else
-        quantize_rowwise_kernel<NT><<<grid, kQThreads, 0, stream>>>(a);
+        quantize_rowwise_kernel<NT, false><<<grid, kQThreads, 0, stream>>>(a);
     return launched();
 }
 
@@ -803,6 +813,6 @@ mx_status mx_quantize_block128(const void* x, int64_t M, int64_t K, int64_t ld_x
 
 void mx_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
 
-void mx_set_quantize_variant(int variant) { g_quant_variant.store(variant == 1 ? 1 : 0); }
+void mx_set_quantize_variant(int variant) { g_quant_variant.store(variant == 1 || variant == 2 ? variant : 0); }
 
 }  // extern "C"

@@ -228,7 +228,11 @@ __device__ __forceinline__ void load_row_tile(const QuantArgs<NT>& a, const Tile
     }
 }
 
-template <int NT>
+// SPLIT == false: the whole next tile is loaded into a second register set at the top of each
+// iteration. SPLIT == true: each half of the next tile is loaded into the registers of the same half
+// of the current tile as soon as that half is encoded (no second set; loads issued later). The host
+// picks SPLIT for long per-CTA tile walks, where it measured faster, and the other form for short ones.
+template <int NT, bool SPLIT>
 __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __grid_constant__ QuantArgs<NT> a) {
     __shared__ __align__(16) uint8_t atom[512];
     const int tid = threadIdx.x;
@@ -236,7 +240,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
     const int64_t per = (a.total_tiles + gridDim.x - 1) / gridDim.x;
     const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
     const int64_t t_end = min(a.total_tiles, t_begin + per);
-    Block32 cur[2], nxt[2];
+    Block32 cur[2], nxt[SPLIT ? 1 : 2];
     TileRef rc, rn;
     if (t_begin < t_end) {
         rc = decode_qtile(a, t_begin);
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
             rn.m0 = static_cast<int64_t>(rn.mt) * kQTile;
             rn.k0 = static_cast<int64_t>(rn.kt) * kQTile;
             rn.full = (rn.m0 + kQTile <= Tn.M) && (rn.k0 + kQTile <= Tn.K);
-            load_row_tile(a, rn, nxt, tid);
+            if constexpr (!SPLIT) load_row_tile(a, rn, nxt, tid);
         }
         const QTensor& T = a.t[rc.i];
         const int kb = tid & 3;
@@ -293,6 +297,12 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
                 }
             }
             atom[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
+            if (SPLIT && t + 1 < t_end) {
+                const QTensor& Tn = a.t[rn.i];
+                const int64_t rown = rn.m0 + h * 64 + (tid >> 2);
+                const int64_t coln = rn.k0 + kb * 32;
+                load_block(Tn, rown, coln, rn.full || (rown < Tn.M && coln < Tn.K), cur[h]);
+            }
         }
         __syncthreads();
         if (a.swz) {
@@ -308,8 +318,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
                     T.s_row[m * kblocks + rc.kt * 4 + q] = atom[(tid & 31) * 16 + (tid >> 5) * 4 + q];
         }
         __syncthreads();
-        cur[0] = nxt[0];
-        cur[1] = nxt[1];
+        if constexpr (!SPLIT) {
+            cur[0] = nxt[0];
+            cur[1] = nxt[1];
+        }
         rc = rn;
     }
 }
@@ -447,10 +459,15 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowcol_kernel(const __g
                 }
                 atom_row[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
             }
+            // Half h of the tile is in shared memory and encoded: the next tile's half h loads into
+            // the same registers and stays in flight through the rest of this tile.
+            if (t + 1 < t_end) {
+                const QTensor& Tn = a.t[rn.i];
+                const int64_t rown = rn.m0 + h * 64 + (tid >> 2);
+                const int64_t coln = rn.k0 + kb * 32;
+                load_block(Tn, rown, coln, rn.full || (rown < Tn.M && coln < Tn.K), cur[h]);
+            }
         }
-        // The tile is in shared memory now: the next tile's loads go into the same registers and
-        // stay in flight through the column pass.
-        if (t + 1 < t_end) load_row_tile(a, rn, cur, tid);
         __syncthreads();
         {
             const int cp = tid & 63;                     // column pair: tile columns 2 cp, 2 cp + 1

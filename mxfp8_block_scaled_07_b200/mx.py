@@ -306,9 +306,10 @@ def set_gemm_variant(variant: int):
     lib().mx_set_gemm_variant(int(variant))
 
 
-QUANT_REGISTERS, QUANT_TMA = 0, 1
+QUANT_REGISTERS, QUANT_TMA, QUANT_SPLIT = 0, 1, 2
 
 
 def set_quantize_variant(variant: int):
-    """0: register-staged quantizer (default); 1: TMA-staged quantizer. Same bytes either way."""
+    """0: register-staged quantizer (default; split loads for long rowwise tile walks); 1: TMA-staged
+    quantizer; 2: register-staged with split loads for every rowwise call. Same bytes in every case."""
     lib().mx_set_quantize_variant(int(variant))

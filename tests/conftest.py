@@ -39,10 +39,10 @@ def gemm_variant(request):
     mx.set_gemm_variant(0)
 
 
-@pytest.fixture(params=[0, 1], ids=["regs", "tma"])
+@pytest.fixture(params=[0, 1, 2], ids=["regs", "tma", "split"])
 def quant_variant(request):
-    """Runs a quantizer test with the register-staged kernel (0, the default) and the TMA-staged
-    kernel (1)."""
+    """Runs a quantizer test with the register-staged kernels (0, the default), the TMA-staged
+    kernel (1) and the register-staged kernels with split loads for every rowwise call (2)."""
     from mxfp8_block_scaled_07_b200 import mx
 
     mx.set_quantize_variant(request.param)
