@@ -1130,7 +1130,7 @@ def main():
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": (round(trec["dram_bytes_per_elem"] * wl.total_elems)
                             if trec else None),
-                "kernel": "quantize_rowwise_kernel<192> (mx_quantize_multi ROWWISE|SWIZZLE, 144 tensors)",
+                "kernel": "quantize_rowwise_kernel<192, split loads> (mx_quantize_multi ROWWISE|SWIZZLE, 144 tensors)",
                 "traffic_source": (trec.get("scaling", "full-launch capture")[:160] if trec else None),
                 "peak_source": f"{peaks['source']} hbm copy (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
                 else "fallback 6.65 TB/s",
