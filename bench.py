@@ -75,6 +75,7 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
+        self.times = []
 
     def __enter__(self):
         try:
@@ -90,6 +91,26 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+            self.times.append(time.monotonic())
+
+    def window(self, t0: float, t1: float) -> dict:
+        """SM clock and power of the samples taken between t0 and t1 (time.monotonic()), or of the
+        nearest sample when the window is shorter than the sampling interval."""
+        rows = []
+        for t, ln in zip(list(self.times), list(self.lines)):
+            parts = [p.strip() for p in ln.split(",")]
+            try:
+                rows.append((t, float(parts[0]), float(parts[2]), parts[4:8]))
+            except (ValueError, IndexError):
+                continue
+        if not rows:
+            return {}
+        inside = [r for r in rows if t0 <= r[0] <= t1] or [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for *_, flags in inside for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "power_w": round(statistics.median(r[2] for r in inside), 1), "reasons": reasons,
+                "samples": len(inside)}
 
     def __exit__(self, *exc):
         if self.proc:
@@ -524,10 +545,12 @@ def flush_l2(buf):
 
 
 def time_gpu(fn, reps, flush_buf, stream):
-    """Median CUDA-event time (ms) of fn over reps runs, L2 flushed before each."""
+    """Median CUDA-event time (ms) of fn over reps runs, L2 flushed before each. The wall-clock
+    window of the runs is kept in time_gpu.window (for the clock samples taken meanwhile)."""
     import torch
 
     times = []
+    t_start = time.monotonic()
     for _ in range(reps):
         flush_l2(flush_buf)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -536,6 +559,7 @@ def time_gpu(fn, reps, flush_buf, stream):
         e1.record(stream)
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
+    time_gpu.window = (t_start, time.monotonic())
     return statistics.median(times)
 
 
@@ -608,10 +632,20 @@ def guarded(fn):
 
 
 def run_secondary(device, peaks, reps=10):
-    """GEMM TFLOP/s on the dense forward, update and MoE configs; quantize GB/s on activations."""
+    """GEMM TFLOP/s on the dense forward, update and MoE configs; quantize GB/s on activations.
+    Each line carries the SM clock and power sampled while it was timed (`clocks`): these lines run
+    after the headline, on a GPU the GEMMs have heated, and a power-capped clock moves them."""
+    with ClockSampler(device.index or 0) as sampler:
+        return _run_secondary(device, peaks, reps, sampler)
+
+
+def _run_secondary(device, peaks, reps, sampler):
     import torch
 
     from mxfp8_block_scaled_07_b200 import mx, synth
+
+    def line_clocks():
+        return {"clocks": sampler.window(*time_gpu.window)}
 
     stream = torch.cuda.current_stream()
     flush = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=device)   # 2 x (2 x L2)
@@ -628,6 +662,7 @@ def run_secondary(device, peaks, reps=10):
         tf = flops / (ms * 1e-3) / 1e12
         rec = {"workload": name, "tflops": round(tf, 1), "ms": round(ms, 4),
                "frac_of_fp8_peak": round(tf / fp8_peak, 3), "frac_of_spec_4500": round(tf / 4500.0, 3)}
+        rec.update(line_clocks())
         rec.update(device_status())
         if lib_fn is not None:
             lib = cublas_line(lib_fn, flops, reps, flush, stream, lib_key)
@@ -647,6 +682,7 @@ def run_secondary(device, peaks, reps=10):
         gbs = nbytes / (ms * 1e-3) / 1e9
         rec = {"workload": name, "gbs": round(gbs, 1), "ms": round(ms, 4),
                "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        rec.update(line_clocks())
         rec.update(device_status())
         out["quantize"].append(rec)
 
@@ -659,6 +695,7 @@ def run_secondary(device, peaks, reps=10):
         ms = time_gpu(fn, reps, flush, stream)
         gbs = (s_raw.numel() + o.numel()) / (ms * 1e-3) / 1e9
         rec = {"workload": name, "gbs": round(gbs, 1), "ms": round(ms, 4), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        rec.update(line_clocks())
         rec.update(device_status())
         out["swizzle"].append(rec)
 

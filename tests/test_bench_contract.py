@@ -64,3 +64,20 @@ def test_breakeven_fit_from_paired_differences():
     assert f["delta_delta_ms"] == pytest.approx(0.010, abs=1e-4)
     assert f["delta_c_us_per_token"] == pytest.approx(0.07, rel=1e-3)
     assert f["m_star_tokens"] == pytest.approx(0.010 / 7.0e-5, rel=1e-3)
+
+
+def test_clock_window_picks_the_samples_of_a_timed_region():
+    """Each secondary line reports the SM clock sampled while it was timed, or the nearest sample
+    when its window is shorter than the sampling interval."""
+    import bench
+
+    cs = bench.ClockSampler(0)
+    flags = "Not Active, Not Active, Not Active"
+    cs.lines = [f"1965, 1965, 700, 0x0, {flags}, Not Active", f"1800, 1965, 950, 0x4, {flags}, Active",
+                f"1700, 1965, 990, 0x4, {flags}, Active"]
+    cs.times = [10.0, 10.1, 10.2]
+    w = cs.window(10.05, 10.25)
+    assert w["sm_mhz"] == 1750 and w["samples"] == 2 and w["reasons"] == ["sw_power_cap"]
+    w = cs.window(9.0, 9.01)
+    assert w["sm_mhz"] == 1965 and w["samples"] == 1 and w["reasons"] == []
+    assert bench.ClockSampler(0).window(0.0, 1.0) == {}
