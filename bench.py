@@ -358,6 +358,52 @@ class SyncWorkload:
             ev_c1.record(stream)
 
 
+def run_fused_sync(wl, stream, step_ms, quant_ms, cmp_ms, steps=10):
+    """The same synchronization check through mx_quantize_compare_multi: one pass quantizes the 144
+    weights (the same grid) and compares what it writes with the sampler's copy, instead of a
+    quantize launch followed by a compare launch that reads the written grid back."""
+    import torch
+
+    from mxfp8_block_scaled_07_b200 import mx
+
+    refs = (mx.GridRef * len(wl.items))()
+    for i, (_, _, _, qs, ss) in enumerate(wl.items):
+        refs[i] = mx.GridRef(qs.data_ptr(), ss.data_ptr())
+    res = torch.empty((2, 2 * len(wl.items)), dtype=torch.int64, device=wl.results.device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def call():
+        st = wl.L.mx_quantize_compare_multi(ctypes.cast(wl.qarr, ctypes.c_void_p), ctypes.cast(refs, ctypes.c_void_p),
+                                            len(wl.items), ctypes.c_void_p(res[0].data_ptr()),
+                                            ctypes.c_void_p(res[1].data_ptr()), sp)
+        if st:
+            raise RuntimeError(f"mx_quantize_compare_multi failed: {st}")
+
+    for _ in range(3):
+        call()
+    mx.device_error()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):          # 28 GB touched per call: far beyond L2, no flush needed
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    fused_ms = e0.elapsed_time(e1) / steps
+    ref_bytes = wl.compare_bytes / 2
+    fused_bytes = wl.quant_bytes + ref_bytes           # BF16 read + grid written + sampler copy read
+    out = {"workload": "qwen3-8b weight sync, 144 tensors: quantize + byte check in one pass "
+                       "(mx_quantize_compare_multi) against the quantize launch + compare launch step",
+           "fused_ms": round(fused_ms, 4), "two_launch_step_ms": round(step_ms, 4),
+           "two_launch_quantize_ms": round(quant_ms, 4), "two_launch_compare_ms": round(cmp_ms, 4),
+           "speedup": round(step_ms / fused_ms, 3),
+           "fused_algorithmic_gb": round(fused_bytes / 1e9, 3),
+           "fused_gbs": round(fused_bytes / (fused_ms * 1e-3) / 1e9, 1),
+           "mismatches": int(res[0].sum().item()),
+           "results_equal_two_launch": bool(torch.equal(res[0], wl.results[0]) and torch.equal(res[1], wl.results[1]))}
+    out.update(device_status())
+    return out
+
+
 def dist_setup(args):
     import torch
 
@@ -1178,6 +1224,9 @@ def main():
     secondary = None
     e2e = None
     cpu = None
+    fused = None
+    if rank == 0 and not args.no_secondary and world == 1:
+        fused = guarded(lambda: run_fused_sync(wl, stream, ms, quant_ms, cmp_ms))
     if not args.no_e2e:                  # every rank: the whole job's end-to-end step
         e2e = aggregate_e2e(pg, run_e2e(wl, args, device), world, wl.step_bytes)
         e2e_err = mx.device_error()
@@ -1190,6 +1239,7 @@ def main():
     # of a multi-GPU run would otherwise wait for them inside a collective.
     if rank == 0 and not args.no_secondary and world == 1:
         secondary = guarded(lambda: run_secondary(device, peaks))
+        secondary["sync_fused"] = fused
         secondary["dense_8192_reference"] = guarded(lambda: run_library_gemm_peak(device))
         secondary["update_breakeven"] = guarded(lambda: run_breakeven(device))
     if rank == 0 and not args.no_cpu_baseline and world == 1:

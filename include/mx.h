@@ -254,6 +254,30 @@ typedef struct {
 mx_status mx_grid_equal_multi(const mx_compare_pair* pairs, int64_t n, unsigned long long* mismatches_dev,
                               long long* first_index_dev, mx_stream stream);
 
+/* The grid a quantization is compared with in mx_quantize_compare_multi. */
+typedef struct {
+    const uint8_t* q;         /* codes [M, K] (device, 16-byte aligned) */
+    const uint8_t* s;         /* scales in the tensor-core layout (device, 16-byte aligned) */
+} mx_grid_ref;
+
+/*
+ * Weight synchronization in one pass (Figure 1: the learner quantizes its weights; Table 11: the
+ * sampler's copy must equal them byte for byte): mx_quantize_multi(tensors, n, MX_ROWWISE |
+ * MX_SWIZZLE) -- the same codes and layout bytes are written to each tensor's q_row / s_row --
+ * fused with the byte comparison of what it writes against refs[i] (e.g. the sampler's copy),
+ * which is read once instead of comparing the written grid in a second pass. Results, on the
+ * device, as mx_grid_equal_multi gives them for the pairs (q_row_i, refs[i].q) and
+ * (s_row_i, refs[i].s): mismatches_dev[2i] / first_index_dev[2i] for the codes (M*K bytes) and
+ * [2i + 1] for the scale layout (mx_swizzled_scale_bytes(M, K/32) bytes); -1 if equal. Entries of
+ * tensors with M == 0 or K == 0 report 0 / -1. `tensors` and `refs` are host memory, read during
+ * the call; each tensor is checked as by mx_quantize (q_col / s_col ignored). Errors: MX_ERR_ARG
+ * (NULL arrays or reference pointers), MX_ERR_ALIGN (reference not 16-byte aligned), and those of
+ * mx_quantize.
+ */
+mx_status mx_quantize_compare_multi(const mx_quant_tensor* tensors, const mx_grid_ref* refs, int64_t n,
+                                    unsigned long long* mismatches_dev, long long* first_index_dev,
+                                    mx_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* mx_status_string(mx_status status);
 

@@ -635,6 +635,52 @@ mx_status mx_grid_equal_multi(const mx_compare_pair* pairs, int64_t n, unsigned 
     return MX_OK;
 }
 
+mx_status mx_quantize_compare_multi(const mx_quant_tensor* tensors, const mx_grid_ref* refs, int64_t n,
+                                    unsigned long long* mismatches_dev, long long* first_index_dev,
+                                    mx_stream stream) {
+    if (n < 0 || (n > 0 && (!tensors || !refs || !mismatches_dev || !first_index_dev))) return MX_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        bool empty = false;
+        if (mx_status st = check_quant_tensor(tensors[i], true, false, &empty)) return st;
+        if (empty) continue;
+        if (!refs[i].q || !refs[i].s) return MX_ERR_ARG;
+        if (!aligned16(refs[i].q) || !aligned16(refs[i].s)) return MX_ERR_ALIGN;
+    }
+    if (n == 0) return MX_OK;
+    const DeviceInfo* d = nullptr;
+    if (mx_status st = check_device(&d)) return st;
+    const int64_t slots = 2 * n;
+    grid_equal_reset_kernel<<<static_cast<int>(std::min<int64_t>(ceil_div(slots, 256), 1024)), 256, 0, stream>>>(
+        mismatches_dev, first_index_dev, static_cast<int>(slots));
+    if (mx_status st = launched()) return st;
+    static thread_local QuantArgs<kQMaxTensors> a;   // ~20 KB: kept off the stack
+    for (int64_t i0 = 0; i0 < n; i0 += kQMaxTensors) {
+        a.n = 0;
+        a.swz = 1;
+        a.total_tiles = 0;
+        a.cmp_counts = mismatches_dev;
+        a.cmp_firsts = first_index_dev;
+        for (int64_t i = i0; i < std::min<int64_t>(n, i0 + kQMaxTensors); ++i) {
+            const mx_quant_tensor& t = tensors[i];
+            if (t.M == 0 || t.K == 0) continue;
+            add_quant_tensor(a, t);
+            QTensor& q = a.t[a.n - 1];
+            q.ref_q = refs[i].q;
+            q.ref_s = refs[i].s;
+            q.res = static_cast<int32_t>(i);
+            q.ref_vec32 = reinterpret_cast<uintptr_t>(refs[i].q) % 32 == 0;
+        }
+        if (a.n == 0) continue;
+        const int64_t grid = std::min<int64_t>(a.total_tiles, int64_t(d->sms) * d->quant_blocks_per_sm[1]);
+        if (a.total_tiles >= kSplitTilesPerCta * grid)
+            quantize_rowwise_kernel<kQMaxTensors, true, true><<<grid, kQThreads, 0, stream>>>(a);
+        else
+            quantize_rowwise_kernel<kQMaxTensors, false, true><<<grid, kQThreads, 0, stream>>>(a);
+        if (mx_status st = launched()) return st;
+    }
+    return MX_OK;
+}
+
 mx_status mx_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb, const uint8_t* sb_swz, int64_t M,
                   int64_t N, int64_t K, void* c, int64_t ld_c, mx_out_dtype out_dtype, mx_stream stream) {
     bool empty = false;

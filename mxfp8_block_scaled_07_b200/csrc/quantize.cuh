@@ -134,6 +134,12 @@ struct QTensor {
     int32_t tiles_m, tiles_k;
     int32_t vec32;            // x rows and q_row 32-byte aligned: 256-bit loads and stores
     int32_t col_vec32;        // q_col 32-byte aligned: 256-bit stores of the transposed copy
+    // Fused comparison (mx_quantize_compare_multi): the grid the codes and swizzled scales are
+    // compared with, and the result slots 2 res (codes) and 2 res + 1 (scales).
+    const uint8_t* ref_q;
+    const uint8_t* ref_s;
+    int32_t res;
+    int32_t ref_vec32;        // ref_q 32-byte aligned: 256-bit loads
 };
 
 struct Block32 {
@@ -163,8 +169,51 @@ struct QuantArgs {
     int n;                    // tensors in this launch
     int swz;                  // write the tensor-core scale layout (else raw scales)
     int64_t total_tiles;
+    unsigned long long* cmp_counts;   // fused comparison: differing bytes per result slot
+    long long* cmp_firsts;            // ... and the index of the first (-1 if none)
     QTensor t[NT];
 };
+
+// Nonzero bytes of x -> 0x01 in that byte.
+__device__ __forceinline__ uint32_t differing_bytes(uint32_t x) {
+    x |= x >> 4;
+    x |= x >> 2;
+    x |= x >> 1;
+    return x & 0x01010101u;
+}
+
+// Adds the differing bytes of `mine` against `ref` (16 bytes at buffer offset `base`) to cnt and
+// lowers first to the smallest differing offset.
+__device__ __forceinline__ void compare16(const uint4& mine, const uint4& ref, int64_t base, unsigned long long& cnt,
+                                          unsigned long long& first) {
+    const uint32_t d[4] = {differing_bytes(mine.x ^ ref.x), differing_bytes(mine.y ^ ref.y),
+                           differing_bytes(mine.z ^ ref.z), differing_bytes(mine.w ^ ref.w)};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (d[k]) {
+            cnt += __popc(d[k]);
+            const unsigned long long idx = static_cast<unsigned long long>(base + 4 * k + (__ffs(d[k]) - 1) / 8);
+            first = idx < first ? idx : first;
+        }
+    }
+}
+
+// Adds one warp's counts to result slot `slot` (only when some lane saw a difference).
+__device__ __forceinline__ void flush_compare(unsigned long long cnt, unsigned long long first,
+                                              unsigned long long* counts, long long* firsts, int slot) {
+    if (__any_sync(0xFFFFFFFFu, cnt != 0)) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
+            const unsigned long long f = __shfl_xor_sync(0xFFFFFFFFu, first, o);
+            first = f < first ? f : first;
+        }
+        if ((threadIdx.x & 31) == 0) {
+            atomicAdd(&counts[slot], cnt);
+            atomicMin(reinterpret_cast<unsigned long long*>(&firsts[slot]), first);
+        }
+    }
+}
 
 struct TileRef {
     int i;                    // tensor index
@@ -232,7 +281,11 @@ __device__ __forceinline__ void load_row_tile(const QuantArgs<NT>& a, const Tile
 // iteration. SPLIT == true: each half of the next tile is loaded into the registers of the same half
 // of the current tile as soon as that half is encoded (no second set; loads issued later). The host
 // picks SPLIT for long per-CTA tile walks, where it measured faster, and the other form for short ones.
-template <int NT, bool SPLIT>
+// CMP == true (weight synchronization, Table 11's byte comparison fused into the quantizer): the
+// codes and the swizzled scale block each tile writes are also compared with a reference grid (the
+// sampler's copy), read once; differing bytes and the first differing offset go to the tensor's
+// result slots, as mx_grid_equal would report them for the written grid.
+template <int NT, bool SPLIT, bool CMP = false>
 __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __grid_constant__ QuantArgs<NT> a) {
     __shared__ __align__(16) uint8_t atom[512];
     const int tid = threadIdx.x;
@@ -241,10 +294,30 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
     const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * per;
     const int64_t t_end = min(a.total_tiles, t_begin + per);
     Block32 cur[2], nxt[SPLIT ? 1 : 2];
+    uint4 ref[2][2];                                     // CMP: the reference codes of this thread's blocks
     TileRef rc, rn;
+    // CMP: reference codes of block h of tile r, loaded one tile ahead like the BF16 input.
+    auto load_ref = [&](const TileRef& r, int h) {
+        const QTensor& Tr = a.t[r.i];
+        const int64_t row = r.m0 + h * 64 + (tid >> 2);
+        const int64_t col = r.k0 + (tid & 3) * 32;
+        if (r.full || (row < Tr.M && col < Tr.K)) {
+            const uint8_t* rq = Tr.ref_q + row * Tr.K + col;
+            if (Tr.ref_vec32) {
+                ld_stream_v8(rq, ref[h][0], ref[h][1]);
+            } else {
+                ref[h][0] = ld_cached_v4(rq);
+                ref[h][1] = ld_cached_v4(rq + 16);
+            }
+        }
+    };
     if (t_begin < t_end) {
         rc = decode_qtile(a, t_begin);
         load_row_tile(a, rc, cur, tid);
+        if constexpr (CMP) {
+            load_ref(rc, 0);
+            load_ref(rc, 1);
+        }
     }
     for (int64_t t = t_begin; t < t_end; ++t) {
         if (t + 1 < t_end) {
@@ -265,6 +338,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
         const QTensor& T = a.t[rc.i];
         const int kb = tid & 3;
         const int64_t col = rc.k0 + kb * 32;
+        unsigned long long ecnt = 0, efirst = ~0ull;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int r = h * 64 + (tid >> 2);           // row inside the tile
@@ -295,6 +369,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
                     reinterpret_cast<uint4*>(q)[0] = o0;
                     reinterpret_cast<uint4*>(q)[1] = o1;
                 }
+                if constexpr (CMP) {
+                    compare16(o0, ref[h][0], row * T.K + col, ecnt, efirst);
+                    compare16(o1, ref[h][1], row * T.K + col + 16, ecnt, efirst);
+                }
             }
             atom[(r & 31) * 16 + (r >> 5) * 4 + kb] = valid ? static_cast<uint8_t>(s) : 0;
             if (SPLIT && t + 1 < t_end) {
@@ -303,12 +381,21 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_rowwise_kernel(const __
                 const int64_t coln = rn.k0 + kb * 32;
                 load_block(Tn, rown, coln, rn.full || (rown < Tn.M && coln < Tn.K), cur[h]);
             }
+            if (CMP && t + 1 < t_end) load_ref(rn, h);
         }
+        if constexpr (CMP) flush_compare(ecnt, efirst, a.cmp_counts, a.cmp_firsts, 2 * T.res);
         __syncthreads();
         if (a.swz) {
-            if (tid < 32)
-                reinterpret_cast<uint4*>(T.s_row + (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512)[tid] =
-                    reinterpret_cast<const uint4*>(atom)[tid];
+            if (tid < 32) {
+                const int64_t soff = (static_cast<int64_t>(rc.mt) * T.tiles_k + rc.kt) * 512;
+                const uint4 mine = reinterpret_cast<const uint4*>(atom)[tid];
+                reinterpret_cast<uint4*>(T.s_row + soff)[tid] = mine;
+                if constexpr (CMP) {
+                    unsigned long long scnt = 0, sfirst = ~0ull;
+                    compare16(mine, ld_cached_v4(T.ref_s + soff + tid * 16), soff + tid * 16, scnt, sfirst);
+                    flush_compare(scnt, sfirst, a.cmp_counts, a.cmp_firsts, 2 * T.res + 1);
+                }
+            }
         } else if (tid < kQTile) {
             const int64_t kblocks = T.K / 32;
             const int64_t m = rc.m0 + tid;

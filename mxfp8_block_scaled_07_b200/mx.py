@@ -31,6 +31,11 @@ class QuantTensor(ctypes.Structure):
                 ("s_col", ctypes.c_void_p)]
 
 
+class GridRef(ctypes.Structure):
+    """mx_grid_ref."""
+    _fields_ = [("q", ctypes.c_void_p), ("s", ctypes.c_void_p)]
+
+
 class ComparePair(ctypes.Structure):
     """mx_compare_pair."""
     _fields_ = [("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("nbytes", ctypes.c_int64)]
@@ -71,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.mx_quantize_multi.restype = I32
     L.mx_grid_equal_multi.argtypes = [P, I64, P, P, P]
     L.mx_grid_equal_multi.restype = I32
+    L.mx_quantize_compare_multi.argtypes = [P, P, I64, P, P, P]
+    L.mx_quantize_compare_multi.restype = I32
     L.mx_status_string.argtypes = [I32]
     L.mx_status_string.restype = ctypes.c_char_p
     L.mx_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -174,6 +181,31 @@ def compare_pair_array(pairs):
         assert a.is_contiguous() and b.is_contiguous() and b.numel() * b.element_size() == n
         arr[i] = ComparePair(a.data_ptr(), b.data_ptr(), n)
     return arr
+
+
+def quantize_compare_multi(xs, refs, outs=None, results=None):
+    """mx_quantize_compare_multi: the rowwise codes and tensor-core scale layout of every BF16
+    tensor in xs (written to outs, as quantize_multi(xs, True, False, True) would), compared byte for
+    byte with refs[i] = (q, s_swizzled) in the same pass. Returns (outs, mismatches, first_index);
+    the last two are int64 device tensors of 2 len(xs) entries: codes then scales per tensor."""
+    n = len(xs)
+    dev = xs[0].device if xs else torch.device("cuda")
+    if outs is None:
+        outs = []
+        for x in xs:
+            M, K = x.shape
+            u8 = dict(dtype=torch.uint8, device=x.device)
+            outs.append((torch.empty((M, K), **u8), torch.empty(swizzled_scale_bytes(M, K // 32), **u8), None, None))
+    if results is None:
+        results = torch.empty((2, max(2 * n, 1)), dtype=torch.int64, device=dev)
+    arr = quant_tensor_array(xs, outs)
+    ref_arr = (GridRef * max(n, 1))()
+    for i, (q, s) in enumerate(refs):
+        ref_arr[i] = GridRef(q.data_ptr(), s.data_ptr())
+    st = lib().mx_quantize_compare_multi(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(ref_arr, ctypes.c_void_p), n,
+                                         _p(results[0]), _p(results[1]), ctypes.c_void_p(_stream(dev)))
+    _check(st, "mx_quantize_compare_multi")
+    return outs, results[0, :2 * n], results[1, :2 * n]
 
 
 def grid_equal_multi(pairs, out=None):

@@ -152,6 +152,30 @@ def test_multi_calls_validate_every_entry(L):
     assert L.mx_grid_equal_multi(None, 0, None, None, None) == 0
 
 
+def test_quantize_compare_multi_validates_before_launching(L):
+    from mxfp8_block_scaled_07_b200 import mx
+
+    P = ctypes.c_void_p
+    good = mx.QuantTensor(0x10000, 64, 64, 64, 0x10000, 0x10000, None, None)
+    arr = (mx.QuantTensor * 2)(good, good)
+    refs = (mx.GridRef * 2)(mx.GridRef(0x10000, 0x10000), mx.GridRef(0x10000, 0x10000))
+    A, R = ctypes.cast(arr, P), ctypes.cast(refs, P)
+    assert L.mx_quantize_compare_multi(None, None, 0, None, None, None) == 0
+    assert L.mx_quantize_compare_multi(A, R, -1, FAKE, FAKE, None) == -1
+    assert L.mx_quantize_compare_multi(A, None, 2, FAKE, FAKE, None) == -1            # no references
+    assert L.mx_quantize_compare_multi(A, R, 2, None, FAKE, None) == -1               # no result array
+    refs[1] = mx.GridRef(0x10000, None)
+    assert L.mx_quantize_compare_multi(A, R, 2, FAKE, FAKE, None) == -1               # 2nd: no reference scales
+    refs[1] = mx.GridRef(0x10008, 0x10000)
+    assert L.mx_quantize_compare_multi(A, R, 2, FAKE, FAKE, None) == -3               # 2nd: misaligned reference
+    refs[1] = mx.GridRef(0x10000, 0x10000)
+    arr[1] = mx.QuantTensor(0x10000, 64, 48, 64, 0x10000, 0x10000, None, None)
+    assert L.mx_quantize_compare_multi(A, R, 2, FAKE, FAKE, None) == -2               # 2nd: K % 32
+    arr[1] = mx.QuantTensor(0x10000, 0, 64, 64, None, None, None, None)
+    refs[1] = mx.GridRef(None, None)                                                   # empty: refs unused
+    assert L.mx_quantize_compare_multi(A, R, 1, FAKE, FAKE, None) != -1
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from mxfp8_block_scaled_07_b200 import mx
 
