@@ -271,8 +271,8 @@ typedef struct {
  * [2i + 1] for the scale layout (mx_swizzled_scale_bytes(M, K/32) bytes); -1 if equal. Entries of
  * tensors with M == 0 or K == 0 report 0 / -1. `tensors` and `refs` are host memory, read during
  * the call; each tensor is checked as by mx_quantize (q_col / s_col ignored). Errors: MX_ERR_ARG
- * (NULL arrays or reference pointers), MX_ERR_ALIGN (reference not 16-byte aligned), and those of
- * mx_quantize.
+ * (NULL arrays or reference pointers, n < 0 or n > 2^30), MX_ERR_ALIGN (reference not 16-byte
+ * aligned), and those of mx_quantize.
  */
 mx_status mx_quantize_compare_multi(const mx_quant_tensor* tensors, const mx_grid_ref* refs, int64_t n,
                                     unsigned long long* mismatches_dev, long long* first_index_dev,

@@ -136,12 +136,18 @@ const DeviceInfo* device_info() {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
         d.status = static_cast<uint32_t*>(p);
-        int split_blocks = 0;
+        // Resident CTAs of the rowwise kernel: the smallest over its load schedules and the fused
+        // comparison forms, which all launch with this grid.
+        int blocks[3] = {0, 0, 0};
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.quant_blocks_per_sm[1],
                                                       quantize_rowwise_kernel<kQMaxTensors, false>, kQThreads, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&split_blocks, quantize_rowwise_kernel<kQMaxTensors, true>,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks[0], quantize_rowwise_kernel<kQMaxTensors, true>,
                                                       kQThreads, 0);
-        d.quant_blocks_per_sm[1] = std::min(d.quant_blocks_per_sm[1], split_blocks);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks[1], quantize_rowwise_kernel<kQMaxTensors, false, true>,
+                                                      kQThreads, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks[2], quantize_rowwise_kernel<kQMaxTensors, true, true>,
+                                                      kQThreads, 0);
+        for (int b : blocks) d.quant_blocks_per_sm[1] = std::min(d.quant_blocks_per_sm[1], b);
         if (d.quant_blocks_per_sm[1] < 1) d.quant_blocks_per_sm[1] = 1;
         d.quant_blocks_per_sm[3] = quant_occupancy<true>();
         if (!qt_setup<true, false>(&d.qt_blocks_per_sm[1]) || !qt_setup<false, true>(&d.qt_blocks_per_sm[2]) ||
@@ -638,7 +644,8 @@ mx_status mx_grid_equal_multi(const mx_compare_pair* pairs, int64_t n, unsigned 
 mx_status mx_quantize_compare_multi(const mx_quant_tensor* tensors, const mx_grid_ref* refs, int64_t n,
                                     unsigned long long* mismatches_dev, long long* first_index_dev,
                                     mx_stream stream) {
-    if (n < 0 || (n > 0 && (!tensors || !refs || !mismatches_dev || !first_index_dev))) return MX_ERR_ARG;
+    if (n < 0 || n > (int64_t(1) << 30) || (n > 0 && (!tensors || !refs || !mismatches_dev || !first_index_dev)))
+        return MX_ERR_ARG;
     for (int64_t i = 0; i < n; ++i) {
         bool empty = false;
         if (mx_status st = check_quant_tensor(tensors[i], true, false, &empty)) return st;
