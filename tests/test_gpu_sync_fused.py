@@ -104,3 +104,24 @@ def test_weight_sync_all_144_tensors_fused():
     c, f = to_np(cnt), to_np(first)
     assert c.sum() == 1 and c[2 * 77] == 1 and f[2 * 77] == 123457
     assert (np.delete(f, 2 * 77) == -1).all()
+
+
+def test_more_tensors_than_one_launch_holds():
+    """200 tensors take two launches (192 + 8): every tensor's results land in its own slots."""
+    g = np.random.default_rng(9)
+    shapes = [(int(g.integers(1, 300)), 32 * int(g.integers(1, 12))) for _ in range(200)]
+    xs = [synth.normal_bf16(sh, seed=100 + i).cuda() for i, sh in enumerate(shapes)]
+    ref = mx.quantize_multi(xs, True, False, True)
+    refs = [(q.clone(), s.clone()) for q, s, _, _ in ref]
+    planted = {3: 0, 191: 5, 192: 0, 199: 7}
+    for i, pos in planted.items():
+        refs[i][0].view(-1)[pos] ^= 1
+    outs, cnt, first = mx.quantize_compare_multi(xs, refs)
+    torch.cuda.synchronize()
+    c, f = to_np(cnt), to_np(first)
+    for i in range(200):
+        want = (1, planted[i]) if i in planted else (0, -1)
+        assert (c[2 * i], f[2 * i]) == want, i
+        assert c[2 * i + 1] == 0 and f[2 * i + 1] == -1, i
+    for (q, s, _, _), (qr, sr, _, _) in zip(outs, ref):
+        assert torch.equal(q, qr) and torch.equal(s, sr)
