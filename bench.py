@@ -1042,7 +1042,8 @@ def run_breakeven(device, reps=20, passes=BREAKEVEN_PASSES):
 
 CASES = ("quant-gate-up", "quant-dy-rowcol", "quant-dy-col", "quant-sync-subset", "quant-fwd-1300", "gemm-fwd-10300",
          "gemm-update-fprop", "gemm-update-dgrad", "gemm-moe-gate-up", "gemm-moe-down", "grid-equal-gate-up",
-         "swizzle-moe-gate-up", "swizzle-moe-down", "block128-pow2-gate-up", "block128-fp32-gate-up")
+         "swizzle-moe-gate-up", "swizzle-moe-down", "block128-pow2-gate-up", "block128-fp32-gate-up",
+         "sync-fused-subset")
 SUBSET_LAYERS = 2      # quant-sync-subset: the first 2 layers' 8 weights (0.39 G elements, ~1.2 GB on the device)
 
 
@@ -1083,6 +1084,15 @@ def run_case(name: str, reps: int):
         q, _, _, _ = mx.quantize(x, True, False)
         q2 = q.clone()
         fn = lambda: mx.grid_equal(q, q2)
+    elif name == "sync-fused-subset":
+        # mx_quantize_compare_multi over the first SUBSET_LAYERS layers' weights against their
+        # sampler copy (here: the learner grid itself), for DRAM-traffic captures.
+        xs = [synth.sync_weight(layer, idx, device=dev) for layer in range(SUBSET_LAYERS) for idx in range(4)]
+        outs = mx.quantize_multi(xs, True, False, True)
+        refs = [(q.clone(), s.clone()) for q, s, _, _ in outs]
+        res = torch.empty((2, 2 * len(xs)), dtype=torch.int64, device=dev)
+        fn = lambda: mx.quantize_compare_multi(xs, refs, outs=outs, results=res)
+        print(json.dumps({"case": name, "tensors": len(xs), "elements": int(sum(x.numel() for x in xs))}))
     elif name.startswith("block128"):
         x = synth.sync_weight(0, 2, device=dev)
         pow2 = name == "block128-pow2-gate-up"
